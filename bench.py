@@ -1,0 +1,402 @@
+"""Benchmark: Hadamard-rotated quantized linear layer on B200.
+
+A step is one pass of the whole hot path over one Llama-70B layer at 4096
+tokens (hidden 8192, FFN 28672, 8 KV heads of 128): forward, dX and dW of the
+seven linear layers q, k, v, o, gate, up, down -- 21 GEMMs, each rotating both
+operands with a block-128 Walsh-Hadamard transform along its contraction
+dimension, quantising per row / column to INT8 and multiplying on the tensor
+cores with a dequantising epilogue.  Inputs are seeded synthetic bf16
+(activations N(0,1) with outlier channels, weights N(0, 0.02^2), output
+gradients N(0, 1e-3^2)); they exceed the 126 MB L2 several times over.
+
+The metric is whole-job throughput in TOPS (2 * M * N * K per GEMM, summed,
+including the rotation and quantisation launches) over the device-timed
+steps; rotate+quantise GB/s and the GEMM kernels' own TOPS are reported beside
+it.  `--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hadamard_rotated_precision_halo_b200 import inputs  # noqa: E402
+
+METRIC = "rotated-qGEMM TOPS & rotate+quant GB/s at Llama shapes vs B200 peak (1 GPU)"
+UNIT = "TOPS"
+BLK = 128
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------- workload
+class LayerStep:
+    """All tensors and launches of one layer step (forward + dX + dW of 7 GEMMs)."""
+
+    def __init__(self, shapes: inputs.LayerShapes, seed: int, device, qtype: int):
+        import hadamard_rotated_precision_halo_b200 as halo
+
+        self.halo = halo
+        self.shapes = shapes
+        self.qtype = qtype
+        self.dev = device
+        self.t = inputs.layer_inputs(shapes, seed, device)
+        t = shapes.tokens
+        self.y, self.dx, self.dw = {}, {}, {}
+        code_dt = torch.int8 if qtype == halo.HALO_Q_INT8 else torch.float8_e4m3fn
+        max_mk = max(t * g.k for g in shapes.gemms)
+        max_nk = max(g.n * g.k for g in shapes.gemms)
+        max_mn = max(t * g.n for g in shapes.gemms)
+        max_vec = max(max(t, g.n, g.k) for g in shapes.gemms)
+        # Code / scale buffers for the two operands of the GEMM in flight.
+        self.qa = torch.empty(max(max_mk, max_mn), dtype=torch.uint8, device=device)
+        self.qb = torch.empty(max(max_nk, max_mk), dtype=torch.uint8, device=device)
+        self.sa = torch.empty(max_vec, dtype=torch.float32, device=device)
+        self.sb = torch.empty(max_vec, dtype=torch.float32, device=device)
+        self.code_dt = code_dt
+        for g in shapes.gemms:
+            self.y[g.name] = torch.empty((t, g.n), dtype=torch.bfloat16, device=device)
+            self.dx[g.name] = torch.empty((t, g.k), dtype=torch.bfloat16, device=device)
+            self.dw[g.name] = torch.empty((g.n, g.k), dtype=torch.float32, device=device)
+        self.ws_fwd = max(halo.halo_workspace_size(t, g.n, g.k, 0) for g in shapes.gemms)
+        self.ws_bwd = max(halo.halo_workspace_size(t, g.n, g.k, 1) for g in shapes.gemms)
+        self.ws = torch.empty(max(self.ws_fwd, self.ws_bwd), dtype=torch.uint8, device=device)
+
+    def ops_per_step(self) -> int:
+        return self.shapes.total_ops()
+
+    def _codes(self, buf, rows, cols):
+        return buf[: rows * cols].view(self.code_dt).view(rows, cols)
+
+    def gemms(self):
+        """The step as (a, a_axis, b, b_axis, m, n, k, out) launch groups, in order."""
+        h = self.halo
+        t = self.shapes.tokens
+        out = []
+        for g in self.shapes.gemms:
+            x, w = self.t["x"][g.x_key], self.t["w"][g.name]
+            out.append(("fwd", g.name, x, h.HALO_AXIS_COLS, w, h.HALO_AXIS_COLS, t, g.n, g.k, self.y[g.name]))
+        for g in self.shapes.gemms:
+            x, w, dy = self.t["x"][g.x_key], self.t["w"][g.name], self.t["dy"][g.name]
+            out.append(("dx", g.name, dy, h.HALO_AXIS_COLS, w, h.HALO_AXIS_ROWS, t, g.k, g.n, self.dx[g.name]))
+            out.append(("dw", g.name, dy, h.HALO_AXIS_ROWS, x, h.HALO_AXIS_ROWS, g.n, g.k, t, self.dw[g.name]))
+        return out
+
+    def run(self, events=None):
+        """One step through the C ABI: per GEMM, rotate+quantise both operands
+        (halo_hadamard_quantize) and multiply (halo_qgemm).  With `events`,
+        record CUDA events around every launch (same stream)."""
+        h = self.halo
+        L = h.lib()
+        stream = torch.cuda.current_stream()
+        sp = h._stream(stream)
+        launches = 0
+        for kind, name, a, a_axis, b, b_axis, m, n, k, c in self.gemms():
+            qa = self._codes(self.qa, a.shape[0], a.shape[1])
+            qb = self._codes(self.qb, b.shape[0], b.shape[1])
+            sa_len = a.shape[0] if a_axis == h.HALO_AXIS_COLS else a.shape[1]
+            sb_len = b.shape[0] if b_axis == h.HALO_AXIS_COLS else b.shape[1]
+            if events is not None:
+                events["rotq"].append(torch.cuda.Event(enable_timing=True))
+                events["rotq"][-1].record(stream)
+            st = L.halo_hadamard_quantize(h._ptr(a), a.shape[0], a.shape[1], a.stride(0), a_axis, BLK, self.qtype,
+                                          h._ptr(qa), qa.stride(0), h._ptr(self.sa), sp)
+            h._check(st, "rotq A")
+            st = L.halo_hadamard_quantize(h._ptr(b), b.shape[0], b.shape[1], b.stride(0), b_axis, BLK, self.qtype,
+                                          h._ptr(qb), qb.stride(0), h._ptr(self.sb), sp)
+            h._check(st, "rotq B")
+            if events is not None:
+                events["gemm"].append(torch.cuda.Event(enable_timing=True))
+                events["gemm"][-1].record(stream)
+            a_major = h.HALO_MAJOR_K if a_axis == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
+            b_major = h.HALO_MAJOR_K if b_axis == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
+            otype = h.HALO_OUT_FP32 if c.dtype == torch.float32 else h.HALO_OUT_BF16
+            st = L.halo_qgemm(h._ptr(qa), h._ptr(self.sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(self.sb),
+                              b_major, qb.stride(0), m, n, k, self.qtype, h._ptr(c), otype, c.stride(0), sp)
+            h._check(st, "qgemm")
+            if events is not None:
+                events["end"].append(torch.cuda.Event(enable_timing=True))
+                events["end"][-1].record(stream)
+            launches += 3
+        return launches
+
+    def rotq_bytes(self) -> int:
+        """Algorithmic bytes of all rotate+quantise launches of one step:
+        bf16 in (2 B) + code out (1 B) per element + one fp32 scale per group."""
+        h = self.halo
+        total = 0
+        for kind, name, a, a_axis, b, b_axis, m, n, k, c in self.gemms():
+            for x, axis in ((a, a_axis), (b, b_axis)):
+                r, cc = x.shape
+                groups = r if axis == h.HALO_AXIS_COLS else cc
+                total += 3 * r * cc + 4 * groups
+        return total
+
+    def gemm_ops(self) -> int:
+        return sum(2 * m * n * k for _, _, _, _, _, _, m, n, k, _ in self.gemms())
+
+
+def e2e_run(step: LayerStep, steps: int):
+    """Same metric end to end through the public linear-layer calls with host
+    buffers: every step copies its inputs from pinned host memory, runs
+    halo_linear_fwd / halo_linear_bwd, and copies all outputs back."""
+    h = step.halo
+    stream = torch.cuda.current_stream()
+    host_in = {key: {n: v.cpu().pin_memory() for n, v in d.items()} for key, d in step.t.items()}
+    host_out = {
+        "y": {n: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for n, v in step.y.items()},
+        "dx": {n: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for n, v in step.dx.items()},
+        "dw": {n: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for n, v in step.dw.items()},
+    }
+    h2d = sum(v.numel() * v.element_size() for d in host_in.values() for v in d.values())
+    d2h = sum(v.numel() * v.element_size() for d in host_out.values() for v in d.values())
+    dev = {key: {n: torch.empty_like(v, device=step.dev) for n, v in d.items()} for key, d in host_in.items()}
+
+    def one():
+        for key, d in host_in.items():
+            for n, v in d.items():
+                dev[key][n].copy_(v, non_blocking=True)
+        t = step.shapes.tokens
+        for g in step.shapes.gemms:
+            x, w = dev["x"][g.x_key], dev["w"][g.name]
+            h.halo_linear_fwd(x, w, BLK, step.qtype, h.HALO_OUT_BF16, y=step.y[g.name], ws=step.ws, stream=stream)
+        for g in step.shapes.gemms:
+            x, w, dy = dev["x"][g.x_key], dev["w"][g.name], dev["dy"][g.name]
+            h.halo_linear_bwd(dy, x, w, BLK, step.qtype, h.HALO_OUT_BF16, h.HALO_OUT_FP32, dx=step.dx[g.name],
+                              dw=step.dw[g.name], ws=step.ws, stream=stream)
+        for key, src in (("y", step.y), ("dx", step.dx), ("dw", step.dw)):
+            for n, v in src.items():
+                host_out[key][n].copy_(v, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    del dev, host_in, host_out
+    return ms, h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU baseline
+def cpu_baseline(seconds_target: float = 15.0):
+    """The oracle as it stands, on a bounded sample of the layer step: the q
+    projection forward (rotate + quantise X rows and all of W_q, integer GEMM,
+    dequantise) restricted to the first R token rows."""
+    import oracle
+
+    shapes = inputs.LLAMA70B_LAYER
+    g = shapes.gemms[0]
+    oracle.build()
+    w = inputs.weights(g.n, g.k, seed=100, device="cpu")
+    rows = 16
+    x = inputs.activations(rows, g.k, seed=101, device="cpu")
+    t0 = time.perf_counter()
+    oracle.linear_fwd(x, w, BLK, oracle.INT8)
+    dt = time.perf_counter() - t0
+    if dt < seconds_target / 3:
+        rows = int(min(512, rows * max(1.0, seconds_target / max(dt, 1e-3) * 0.8)))
+        x = inputs.activations(rows, g.k, seed=101, device="cpu")
+        t0 = time.perf_counter()
+        oracle.linear_fwd(x, w, BLK, oracle.INT8)
+        dt = time.perf_counter() - t0
+    ops = 2 * rows * g.n * g.k
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"q-projection forward, {rows} of {shapes.tokens} token rows x W[{g.n},{g.k}], "
+                      f"INT8, block 128 ({dt:.1f} s)"}
+
+
+# ------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="halo", choices=["halo", "reference"])
+    ap.add_argument("--qtype", default="int8", choices=["int8", "e4m3"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    shapes = inputs.LLAMA70B_LAYER
+    config = {"workload": "llama70b_layer_fwd_bwd", "tokens": shapes.tokens, "hidden": shapes.hidden,
+              "ffn": shapes.ffn, "kv": shapes.kv, "gemms": 21, "block": BLK, "qtype": args.qtype,
+              "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = cpu_baseline()
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import hadamard_rotated_precision_halo_b200 as halo
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    qtype = halo.HALO_Q_INT8 if args.qtype == "int8" else halo.HALO_Q_E4M3
+    step = LayerStep(shapes, seed=4 + rank, device=device, qtype=qtype)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        step.run()
+    torch.cuda.synchronize()
+    st, site = halo.halo_device_error()
+    if st != halo.HALO_OK:
+        raise RuntimeError(f"device error after warm-up at site {site:#x}")
+
+    events = {"rotq": [], "gemm": [], "end": []}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        launches = 0
+        for _ in range(args.steps):
+            launches += step.run(events)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    st, site = halo.halo_device_error()
+    if st != halo.HALO_OK:
+        raise RuntimeError(f"device error in the timed region at site {site:#x}")
+
+    rotq_ms = sum(a.elapsed_time(b) for a, b in zip(events["rotq"], events["gemm"]))
+    gemm_ms = sum(a.elapsed_time(b) for a, b in zip(events["gemm"], events["end"]))
+    n_gemm = len(events["gemm"])
+    ops_step = step.ops_per_step()
+    ms_step = ms_total / args.steps
+    value = ops_step * args.steps * world / (ms_total * 1e-3) / 1e12
+    gemm_tops = step.gemm_ops() * args.steps / (gemm_ms * 1e-3) / 1e12
+    rotq_gbs = step.rotq_bytes() * args.steps / (rotq_ms * 1e-3) / 1e9
+    pk = peaks()
+    # INT8 / FP8 dense peak: the measured bf16 cuBLAS figure times the nominal
+    # 8-bit : bf16 ratio (4.5 : 2.25); sustained figure, the GEMMs run inside a long step.
+    peak8 = 2.0 * pk["bf16_sustained"]
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8" if qtype == halo.HALO_Q_INT8 else "e4m3",
+            "data": "synthetic", "config": config,
+            "gpu_launches": launches,
+            "roofline": {"bound": "tensor", "kernel": "qgemm_kernel", "achieved": gemm_tops, "peak": peak8,
+                         "unit": "TFLOP/s", "frac": gemm_tops / peak8, "traffic": None,
+                         "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']})",
+                         "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
+            "rotq": {"gbs": rotq_gbs, "peak_gbs": pk["hbm_gbs"], "frac": rotq_gbs / pk["hbm_gbs"],
+                     "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps},
+            "clocks": clocks.summary()}
+
+    if rank == 0 and not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_run(step, steps=2)
+        line["e2e"] = {"value": ops_step / (e2e_ms * 1e-3) / 1e12 * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

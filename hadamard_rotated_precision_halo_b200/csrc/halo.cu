@@ -1,0 +1,502 @@
+// halo.cu -- C ABI (include/halo.h): validation, tensor-map encoding and launch
+// orchestration for the rotate+quantise kernels and the tcgen05 GEMM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/halo.h"
+#include "qgemm.cuh"
+#include "rotq.cuh"
+
+using namespace halo;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sm_count = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+halo_status_t cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return HALO_ERR_CUDA;
+}
+
+#define HALO_CUDA(call)                         \
+  do {                                          \
+    cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+template <typename K>
+cudaError_t set_smem_attr(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+// One-time per-device set-up: architecture check, SM count, kernel attributes,
+// driver entry point for tensor-map encoding.
+halo_status_t device_setup(int* dev_out) {
+  int dev = 0;
+  HALO_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return HALO_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  DeviceInfo& d = g_dev[dev];
+  if (d.ready) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (d.ready) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+  int major = 0, minor = 0;
+  HALO_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  HALO_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  HALO_CUDA(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev));
+  d.supported = (major == 10 && minor == 0);
+  if (d.supported) {
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      HALO_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn) return HALO_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    const size_t big = 227 * 1024;
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 0>, big));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 1>, big));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 0>, big));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 1>, big));
+    HALO_CUDA(set_smem_attr(rotq_cols_kernel<0>, big));
+    HALO_CUDA(set_smem_attr(rotq_cols_kernel<1>, big));
+    HALO_CUDA(set_smem_attr(qgemm_kernel<0>, kGemmSmemBytes));
+    HALO_CUDA(set_smem_attr(qgemm_kernel<1>, kGemmSmemBytes));
+  }
+  d.ready = true;
+  return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+                     const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides_bytes, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return HALO_ERR_CUDA;
+  }
+  return HALO_OK;
+}
+
+// ------------------------------------------------------------------------ rotq launches
+halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
+                               void* q, int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
+  const int nb = static_cast<int>(cols / 128);
+  // About 128 chunks per tile; a tile always holds whole rows (for blk 256, nb
+  // is even, so the two chunks of a block sit on adjacent lanes).
+  const int nr = std::max(1, 128 / nb);
+  const int active = nr * nb;
+  const int threads = (active + 31) / 32 * 32;
+  const int num_tiles = static_cast<int>((rows + nr - 1) / nr);
+
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(nb), static_cast<cuuint32_t>(nr)};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[3] = {kRowsOutSlot, static_cast<cuuint32_t>(nb), static_cast<cuuint32_t>(nr)};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  const size_t in_stride = (static_cast<size_t>(active) * kRowsInSlot + 127) & ~size_t(127);
+  const size_t out_stride = (static_cast<size_t>(active) * kRowsOutSlot + 127) & ~size_t(127);
+  const size_t smem = 2 * in_stride + 2 * out_stride + 128;  // + alignment slack
+
+  RotqRowsParams p;
+  p.scales = scales;
+  p.rows = rows;
+  p.nb = nb;
+  p.nr = nr;
+  p.num_tiles = num_tiles;
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(static_cast<double>(blk))));
+
+  void (*kern)(const CUtensorMap, const CUtensorMap, RotqRowsParams) = nullptr;
+  if (blk == 128)
+    kern = qtype == HALO_Q_INT8 ? rotq_rows_kernel<128, 0> : rotq_rows_kernel<128, 1>;
+  else
+    kern = qtype == HALO_Q_INT8 ? rotq_rows_kernel<256, 0> : rotq_rows_kernel<256, 1>;
+  int per_sm = 0;
+  HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
+  if (per_sm < 1) per_sm = 1;
+  const int grid = static_cast<int>(std::min<int64_t>(num_tiles, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
+  kern<<<grid, threads, smem, stream>>>(tm_x, tm_q, p);
+  HALO_CUDA(cudaGetLastError());
+  return HALO_OK;
+}
+
+halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
+                               int64_t ld_q, float* scales, cudaStream_t stream) {
+  const int nblocks = static_cast<int>(rows / 128);
+  int cl = 8;
+  while (cl > 1 && cl > nblocks) cl /= 2;
+  const int warps = std::max(1, std::min(4, (nblocks + cl - 1) / cl));
+  const int strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
+
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  RotqColsParams p;
+  p.scales = scales;
+  p.cols = cols;
+  p.nblocks = nblocks;
+  p.warps = warps;
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  const size_t smem = static_cast<size_t>(warps) * (kColsStages * kColsInBytes + 2 * kColsOutBytes) + 128;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cl, strips, 1);
+  cfg.blockDim = dim3(32 * warps, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (qtype == HALO_Q_INT8)
+    HALO_CUDA(cudaLaunchKernelEx(&cfg, rotq_cols_kernel<0>, tm_x, tm_q, p));
+  else
+    HALO_CUDA(cudaLaunchKernelEx(&cfg, rotq_cols_kernel<1>, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
+// ------------------------------------------------------------------------ GEMM launch
+halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_a, const void* b, const float* sb,
+                           int b_mn, int64_t ld_b, int64_t m, int64_t n, int64_t k, int qtype, void* c, int otype,
+                           int64_t ld_c, cudaStream_t stream, int dev) {
+  CUtensorMap tm_a, tm_b;
+  const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  {
+    cuuint64_t dims[2];
+    if (a_mn) {
+      dims[0] = static_cast<cuuint64_t>(m);
+      dims[1] = static_cast<cuuint64_t>(k);
+    } else {
+      dims[0] = static_cast<cuuint64_t>(k);
+      dims[1] = static_cast<cuuint64_t>(m);
+    }
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_a)};
+    cuuint32_t box[2] = {128, 128};
+    halo_status_t st = encode(&tm_a, dt, 2, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2];
+    cuuint32_t box[2];
+    if (b_mn) {
+      dims[0] = static_cast<cuuint64_t>(n);
+      dims[1] = static_cast<cuuint64_t>(k);
+      box[0] = 128;
+      box[1] = 128;
+    } else {
+      dims[0] = static_cast<cuuint64_t>(k);
+      dims[1] = static_cast<cuuint64_t>(n);
+      box[0] = 128;
+      box[1] = 256;
+    }
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_b)};
+    halo_status_t st = encode(&tm_b, dt, 2, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != HALO_OK) return st;
+  }
+  GemmParams p;
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.tiles_m = static_cast<int>((m + kGemmBM - 1) / kGemmBM);
+  p.tiles_n = static_cast<int>((n + kGemmBN - 1) / kGemmBN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
+  // Instruction descriptor: D format (bits 4-5), A/B formats (7-9, 10-12),
+  // A/B major (15, 16), N >> 3 (17-22), M >> 4 (24-28).
+  uint32_t idesc = 0;
+  if (qtype == HALO_Q_INT8)
+    idesc |= (2u << 4) | (1u << 7) | (1u << 10);  // s32 accumulate, signed 8-bit A and B
+  else
+    idesc |= (1u << 4);                           // f32 accumulate, E4M3 A and B
+  idesc |= static_cast<uint32_t>(a_mn) << 15;
+  idesc |= static_cast<uint32_t>(b_mn) << 16;
+  idesc |= static_cast<uint32_t>(kGemmBN >> 3) << 17;
+  idesc |= static_cast<uint32_t>(kGemmBM >> 4) << 24;
+  p.idesc = idesc;
+  p.sa = sa;
+  p.sb = sb;
+  p.c = c;
+  p.ldc = ld_c;
+  p.out_bf16 = otype == HALO_OUT_BF16;
+  const int grid = std::min(p.num_tiles, g_dev[dev].sm_count);
+  if (qtype == HALO_Q_INT8)
+    qgemm_kernel<0><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+  else
+    qgemm_kernel<1><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+  HALO_CUDA(cudaGetLastError());
+  return HALO_OK;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool valid_qtype(int q) { return q == HALO_Q_INT8 || q == HALO_Q_E4M3; }
+bool valid_otype(int o) { return o == HALO_OUT_FP32 || o == HALO_OUT_BF16; }
+
+halo_status_t check_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int axis, int blk,
+                                      int qtype, const void* q, int64_t ld_q, const float* scales) {
+  if (!x || !q || !scales) return HALO_ERR_NULL;
+  if (!valid_qtype(qtype) || (axis != HALO_AXIS_COLS && axis != HALO_AXIS_ROWS)) return HALO_ERR_DTYPE;
+  if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
+  if (axis == HALO_AXIS_ROWS && blk != 128) return HALO_ERR_BLOCK;
+  if (rows <= 0 || cols <= 0 || ld_x < cols || ld_q < cols) return HALO_ERR_SHAPE;
+  if (axis == HALO_AXIS_COLS && (cols % blk != 0 || cols > 32768)) return HALO_ERR_SHAPE;
+  if (axis == HALO_AXIS_ROWS && (rows % blk != 0 || cols % 8 != 0)) return HALO_ERR_SHAPE;
+  if (rows > (int64_t(1) << 31) - 1 || cols > (int64_t(1) << 31) - 1) return HALO_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(scales) || (ld_x * 2) % 16 != 0 || ld_q % 16 != 0)
+    return HALO_ERR_ALIGN;
+  return HALO_OK;
+}
+
+halo_status_t check_qgemm(const void* a, const float* sa, int a_major, int64_t ld_a, const void* b,
+                          const float* sb, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k, int qtype,
+                          const void* c, int otype, int64_t ld_c) {
+  if (!a || !sa || !b || !sb || !c) return HALO_ERR_NULL;
+  if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
+  if ((a_major != HALO_MAJOR_K && a_major != HALO_MAJOR_MN) || (b_major != HALO_MAJOR_K && b_major != HALO_MAJOR_MN))
+    return HALO_ERR_DTYPE;
+  if (m <= 0 || n <= 0 || k <= 0) return HALO_ERR_SHAPE;
+  if (m > (int64_t(1) << 31) - 1 || n > (int64_t(1) << 31) - 1) return HALO_ERR_SHAPE;
+  if (qtype == HALO_Q_INT8 && k > 133144) return HALO_ERR_SHAPE;
+  if (k > (int64_t(1) << 31) - 1) return HALO_ERR_SHAPE;
+  if (ld_a < (a_major == HALO_MAJOR_K ? k : m) || ld_b < (b_major == HALO_MAJOR_K ? k : n) || ld_c < n)
+    return HALO_ERR_SHAPE;
+  const int64_t esz = otype == HALO_OUT_FP32 ? 4 : 2;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c) || !aligned16(sa) || !aligned16(sb) || ld_a % 16 != 0 ||
+      ld_b % 16 != 0 || (ld_c * esz) % 16 != 0)
+    return HALO_ERR_ALIGN;
+  return HALO_OK;
+}
+
+// Workspace layout (each region 256-byte aligned):
+//   fwd: Xq[M*K] Wq[N*K] sx[M] sw[N]
+//   bwd: dYq_rows[M*N] Wq_cols[N*K] s_dy_rows[M] s_w_cols[K]
+//        dYq_cols[M*N] Xq_cols[M*K] s_dy_cols[N] s_x_cols[K]
+struct WsLayout {
+  size_t off[8];
+  size_t total;
+};
+
+WsLayout ws_layout(int64_t m, int64_t n, int64_t k, int which) {
+  WsLayout L = {};
+  size_t sizes[8];
+  int cnt;
+  if (which == 0) {
+    sizes[0] = size_t(m) * k;
+    sizes[1] = size_t(n) * k;
+    sizes[2] = size_t(m) * 4;
+    sizes[3] = size_t(n) * 4;
+    cnt = 4;
+  } else {
+    sizes[0] = size_t(m) * n;
+    sizes[1] = size_t(n) * k;
+    sizes[2] = size_t(m) * 4;
+    sizes[3] = size_t(k) * 4;
+    sizes[4] = size_t(m) * n;
+    sizes[5] = size_t(m) * k;
+    sizes[6] = size_t(n) * 4;
+    sizes[7] = size_t(k) * 4;
+    cnt = 8;
+  }
+  size_t off = 0;
+  for (int i = 0; i < cnt; ++i) {
+    L.off[i] = off;
+    off = align_up(off + sizes[i], 256);
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* halo_status_string(int status) {
+  switch (status) {
+    case HALO_OK: return "HALO_OK";
+    case HALO_ERR_NULL: return "HALO_ERR_NULL: a required pointer is NULL";
+    case HALO_ERR_SHAPE: return "HALO_ERR_SHAPE: invalid or unsupported size";
+    case HALO_ERR_BLOCK: return "HALO_ERR_BLOCK: unsupported Hadamard block size";
+    case HALO_ERR_ALIGN: return "HALO_ERR_ALIGN: pointer or stride alignment";
+    case HALO_ERR_DTYPE: return "HALO_ERR_DTYPE: unknown qtype / otype / axis / major";
+    case HALO_ERR_WORKSPACE: return "HALO_ERR_WORKSPACE: workspace missing or too small";
+    case HALO_ERR_CUDA: return "HALO_ERR_CUDA: a CUDA call failed";
+    case HALO_ERR_TIMEOUT: return "HALO_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    case HALO_ERR_UNSUPPORTED: return "HALO_ERR_UNSUPPORTED: device is not sm_100 (B200)";
+    default: return "HALO: unknown status";
+  }
+}
+
+int halo_last_cuda_error(void) { return g_last_cuda_error; }
+
+halo_status_t halo_device_error(int* where) {
+  HALO_CUDA(cudaDeviceSynchronize());
+  unsigned int site = 0, zero = 0;
+  HALO_CUDA(cudaMemcpyFromSymbol(&site, g_error_site, sizeof(site)));
+  if (site != 0) HALO_CUDA(cudaMemcpyToSymbol(g_error_site, &zero, sizeof(zero)));
+  if (where) *where = static_cast<int>(site);
+  return site ? HALO_ERR_TIMEOUT : HALO_OK;
+}
+
+size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which) {
+  if (m <= 0 || n <= 0 || k <= 0 || (which != 0 && which != 1)) return 0;
+  return ws_layout(m, n, k, which).total;
+}
+
+halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int axis,
+                                     int blk, int qtype, void* q_out, int64_t ld_q, float* scales_out,
+                                     void* stream) {
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, axis, blk, qtype, q_out, ld_q, scales_out);
+  if (st != HALO_OK) return st;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (axis == HALO_AXIS_COLS) return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, qtype, q_out, ld_q, scales_out, s, dev);
+  return launch_rotq_cols(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, s);
+}
+
+halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,
+                         const float* s_b, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k, int qtype,
+                         void* c, int otype, int64_t ld_c, void* stream) {
+  halo_status_t st = check_qgemm(a_q, s_a, a_major, ld_a, b_q, s_b, b_major, ld_b, m, n, k, qtype, c, otype, ld_c);
+  if (st != HALO_OK) return st;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  return launch_qgemm(a_q, s_a, a_major, ld_a, b_q, s_b, b_major, ld_b, m, n, k, qtype, c, otype, ld_c,
+                      static_cast<cudaStream_t>(stream), dev);
+}
+
+halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k, int blk,
+                              int qtype, void* y, int otype, void* ws, size_t ws_bytes, void* stream) {
+  if (!x_bf16 || !w_bf16 || !y) return HALO_ERR_NULL;
+  if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
+  if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
+  if (m <= 0 || n <= 0 || k <= 0 || k % blk != 0 || k > 32768) return HALO_ERR_SHAPE;
+  if (!ws) return HALO_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(m, n, k, 0);
+  if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
+  const int64_t esz = otype == HALO_OUT_FP32 ? 4 : 2;
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y) || !aligned16(ws) || (n * esz) % 16 != 0)
+    return HALO_ERR_ALIGN;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint8_t* xq = w8 + L.off[0];
+  uint8_t* wq = w8 + L.off[1];
+  float* sx = reinterpret_cast<float*>(w8 + L.off[2]);
+  float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
+  halo_status_t st;
+  if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_COLS, blk, qtype, xq, k, sx, stream)) != HALO_OK) return st;
+  if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_COLS, blk, qtype, wq, k, sw, stream)) != HALO_OK) return st;
+  return halo_qgemm(xq, sx, HALO_MAJOR_K, k, wq, sw, HALO_MAJOR_K, k, m, n, k, qtype, y, otype, n, stream);
+}
+
+halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
+                              int64_t k, int blk, int qtype, void* dx, int otype_dx, void* dw, int otype_dw,
+                              void* ws, size_t ws_bytes, void* stream) {
+  if (!dy_bf16 || (!dx && !dw)) return HALO_ERR_NULL;
+  if (dx && !w_bf16) return HALO_ERR_NULL;
+  if (dw && !x_bf16) return HALO_ERR_NULL;
+  if (!valid_qtype(qtype) || (dx && !valid_otype(otype_dx)) || (dw && !valid_otype(otype_dw))) return HALO_ERR_DTYPE;
+  if (blk != 128) return HALO_ERR_BLOCK;
+  if (m <= 0 || n <= 0 || k <= 0) return HALO_ERR_SHAPE;
+  if (dx && (n % blk != 0 || n > 32768 || k % 16 != 0)) return HALO_ERR_SHAPE;
+  if (dw && (m % blk != 0 || n % 16 != 0 || k % 16 != 0)) return HALO_ERR_SHAPE;
+  if (!ws) return HALO_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(m, n, k, 1);
+  if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
+  if (!aligned16(dy_bf16) || (x_bf16 && !aligned16(x_bf16)) || (w_bf16 && !aligned16(w_bf16)) ||
+      (dx && !aligned16(dx)) || (dw && !aligned16(dw)) || !aligned16(ws))
+    return HALO_ERR_ALIGN;
+  if (dx && (k * (otype_dx == HALO_OUT_FP32 ? 4 : 2)) % 16 != 0) return HALO_ERR_ALIGN;
+  if (dw && (k * (otype_dw == HALO_OUT_FP32 ? 4 : 2)) % 16 != 0) return HALO_ERR_ALIGN;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  halo_status_t st;
+  if (dx) {
+    uint8_t* dyq = w8 + L.off[0];
+    uint8_t* wq = w8 + L.off[1];
+    float* sdy = reinterpret_cast<float*>(w8 + L.off[2]);
+    float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
+    // dX[M,K] = dY[M,N] W[N,K]: contraction over N.
+    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, qtype, dyq, n, sdy, stream)) != HALO_OK)
+      return st;
+    if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_ROWS, blk, qtype, wq, k, sw, stream)) != HALO_OK)
+      return st;
+    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_K, n, wq, sw, HALO_MAJOR_MN, k, m, k, n, qtype, dx, otype_dx, k,
+                         stream)) != HALO_OK)
+      return st;
+  }
+  if (dw) {
+    uint8_t* dyq = w8 + L.off[4];
+    uint8_t* xq = w8 + L.off[5];
+    float* sdy = reinterpret_cast<float*>(w8 + L.off[6]);
+    float* sx = reinterpret_cast<float*>(w8 + L.off[7]);
+    // dW[N,K] = dY^T[N,M] X[M,K]: contraction over M (tokens).
+    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, qtype, dyq, n, sdy, stream)) != HALO_OK)
+      return st;
+    if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_ROWS, blk, qtype, xq, k, sx, stream)) != HALO_OK)
+      return st;
+    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_MN, n, xq, sx, HALO_MAJOR_MN, k, n, k, m, qtype, dw, otype_dw, k,
+                         stream)) != HALO_OK)
+      return st;
+  }
+  return HALO_OK;
+}
+
+}  // extern "C"

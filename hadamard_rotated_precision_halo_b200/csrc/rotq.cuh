@@ -1,0 +1,442 @@
+// rotq.cuh -- fused block Walsh-Hadamard rotation + absmax + symmetric quantisation.
+//
+// Two kernels, one per rotation axis of a bf16 matrix X[rows, cols]:
+//
+//   rotq_rows_kernel  rotate along the contiguous dimension (blocks of 128 or
+//                     256 consecutive elements of a row), one scale per row.
+//   rotq_cols_kernel  rotate along dimension 0 (blocks of 128 consecutive rows
+//                     of a column), one scale per column.
+//
+// Both compute, for every group g (a row or a column),
+//     u      = H_blk x            (unnormalised Sylvester transform, fp32)
+//     amax_g = max |u|            (over the whole group)
+//     s_g    = amax_g / (qmax sqrt(blk))        -> scale of the normalised value
+//     q      = round_half_even(u * qmax / amax_g)   (INT8; |q| <= 127 by construction)
+//            | e4m3_rn_satfinite(u * qmax / amax_g) (E4M3)
+// which equals quantising the normalised rotation H_blk x / sqrt(blk) with
+// scale s_g: the 1/sqrt(blk) factor cancels in the codes and only enters s_g.
+// Walsh-Hadamard transform and quantiser: QWHA page sec. 2.1-2.2; INT8 / FP8:
+// HALO paper page, "key design"; block-local rotation: HALO blog page sec. 5.
+//
+// Memory path (HBM-bound): one TMA read of the bf16 input, one TMA write of the
+// 1-byte codes, one fp32 scale per group.  Every FWHT butterfly runs in
+// registers (packed f32x2 adds), no data crosses threads except the top stage
+// of a 256-block (one shuffle per element).
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "ptx.cuh"
+
+namespace halo {
+
+enum : unsigned int {
+  kSiteRotqRowsLoad = 0x101,
+  kSiteRotqColsLoad = 0x201,
+};
+
+// Per-thread slot sizes in shared memory for rotq_rows: 128 bf16 (256 B) plus
+// 16 B of padding, and 128 code bytes plus 16 B of padding.  The padding makes
+// the per-thread 16-byte accesses of a quarter warp hit eight distinct bank
+// groups.
+constexpr int kRowsInSlot = 272;   // bytes (136 bf16)
+constexpr int kRowsOutSlot = 144;  // bytes
+
+struct RotqRowsParams {
+  float* scales;
+  int64_t rows;
+  int nb;          // 128-element chunks per row (cols / 128)
+  int nr;          // rows per tile
+  int num_tiles;   // ceil(rows / nr)
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(blk))
+};
+
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// In-register unnormalised Walsh-Hadamard transform of 128 values held as 64
+// float2 pairs (v[i] = elements 2i, 2i+1), natural Sylvester order.
+__device__ __forceinline__ void fwht128_pairs(float2 (&v)[64]) {
+  // h = 1: butterflies inside each pair.
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float a = v[i].x, b = v[i].y;
+    v[i] = make_float2(a + b, a - b);
+  }
+  // h = 2 .. 64: pair i with pair i + h/2.
+#pragma unroll
+  for (int hp = 1; hp < 64; hp *= 2) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      if ((i & hp) == 0) {
+        const float2 a = v[i], b = v[i + hp];
+        v[i] = f2_add(a, b);
+        v[i + hp] = f2_sub(a, b);
+      }
+    }
+  }
+}
+
+// Round-half-even of t (|t| <= 2^22) to an int8 code in the low byte of the
+// returned word: adding 1.5 * 2^23 puts the rounded integer into the low
+// mantissa bits (round-to-nearest-even of the fused multiply-add).
+__device__ __forceinline__ uint32_t q_int8_bits(float u, float r) {
+  return __float_as_uint(__fmaf_rn(u, r, 12582912.0f));
+}
+
+__device__ __forceinline__ uint32_t pack4_int8(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  const uint32_t lo = __byte_perm(b0, b1, 0x0040);
+  const uint32_t hi = __byte_perm(b2, b3, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// ------------------------------------------------------------------------------------------
+// rotq_rows: one thread owns one 128-element chunk of one row.  A tile is `nr`
+// whole rows (nr * nb chunks <= blockDim.x).  The tile arrives by one 3-D TMA
+// load of the view [rows][nb][128] with a 136-element box along the innermost
+// dimension: the 8 elements past each chunk fall outside the tensor, read as
+// zeros and give the padded slot layout for free.  Codes leave the same way
+// (144-byte box, the out-of-range tail is not written).
+// ------------------------------------------------------------------------------------------
+template <int BLK, int QT>
+__global__ void __launch_bounds__(256, 1)
+    rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                     RotqRowsParams p) {
+  constexpr int kStages = 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t full_bar[kStages];
+  __shared__ uint32_t s_amax[2][256];
+
+  const int tid = threadIdx.x;
+  const int active = p.nr * p.nb;
+  const uint32_t in_bytes = static_cast<uint32_t>(active) * kRowsInSlot;
+  const uint32_t in_stride = (in_bytes + 127u) & ~127u;
+  const uint32_t out_bytes = static_cast<uint32_t>(active) * kRowsOutSlot;
+  const uint32_t out_stride = (out_bytes + 127u) & ~127u;
+  uint8_t* s_in = smem;
+  uint8_t* s_out = smem + kStages * in_stride;
+
+  const int my_row = tid / p.nb;
+  const int my_chunk = tid - my_row * p.nb;
+  const bool is_active = tid < active;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full_bar[s], 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_q);
+  }
+  for (int i = tid; i < 2 * 256; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
+  __syncthreads();
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      const int tile = blockIdx.x + s * gridDim.x;
+      if (tile < p.num_tiles) {
+        mbar_arrive_expect_tx(&full_bar[s], in_bytes);
+        tma_load_3d(s_in + s * in_stride, &tm_x, &full_bar[s], 0, 0, tile * p.nr);
+      }
+    }
+  }
+
+  uint32_t it = 0;
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+    const int s = it % kStages;
+    const uint32_t ph = (it / kStages) & 1u;
+    const int par = it & 1;
+    const bool ok = mbar_wait(&full_bar[s], ph, kSiteRotqRowsLoad);
+    if (__syncthreads_or(!ok)) break;
+
+    uint4 raw[16];
+    if (is_active) {
+      const uint4* src = reinterpret_cast<const uint4*>(s_in + s * in_stride + tid * kRowsInSlot);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) raw[k] = src[k];
+    }
+    __syncthreads();  // stage s fully consumed; code buffer `par` free once the wait below returns
+    if (tid == 0) {
+      const int next = tile + kStages * gridDim.x;
+      if (next < p.num_tiles) {
+        mbar_arrive_expect_tx(&full_bar[s], in_bytes);
+        tma_load_3d(s_in + s * in_stride, &tm_x, &full_bar[s], 0, 0, next * p.nr);
+      }
+      bulk_wait_read<1>();
+    }
+    for (int i = tid; i < p.nr; i += blockDim.x) s_amax[par ^ 1][i] = 0u;
+
+    float2 v[64];
+    float amax = 0.f;
+    if (is_active) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        v[4 * k + 0] = bf16x2_to_f2(raw[k].x);
+        v[4 * k + 1] = bf16x2_to_f2(raw[k].y);
+        v[4 * k + 2] = bf16x2_to_f2(raw[k].z);
+        v[4 * k + 3] = bf16x2_to_f2(raw[k].w);
+      }
+      fwht128_pairs(v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
+    }
+    if (BLK == 256) {
+      // Top stage of the 256-point transform: chunk pairs (2j, 2j+1) of a row
+      // sit on adjacent lanes.  Lower half keeps a + b, upper half a - b.
+      // Every lane of the warp takes part (idle lanes carry zeros).
+      const bool upper = (my_chunk & 1) != 0;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float2 o;
+        o.x = __shfl_xor_sync(0xffffffffu, v[i].x, 1);
+        o.y = __shfl_xor_sync(0xffffffffu, v[i].y, 1);
+        v[i] = upper ? f2_sub(o, v[i]) : f2_add(v[i], o);
+      }
+    }
+    if (is_active) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      atomicMax(&s_amax[par][my_row], __float_as_uint(amax));
+    }
+    __syncthreads();
+
+    if (is_active) {
+      const float row_amax = __uint_as_float(s_amax[par][my_row]);
+      const float r = row_amax > 0.f ? __fdiv_rn(p.qmax, row_amax) : 0.f;
+      const int64_t grow = static_cast<int64_t>(tile) * p.nr + my_row;
+      if (my_chunk == 0 && grow < p.rows) p.scales[grow] = row_amax * p.scale_mult;
+      uint4* dst = reinterpret_cast<uint4*>(s_out + par * out_stride + tid * kRowsOutSlot);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 a = v[8 * k + 2 * j];
+          const float2 b = v[8 * k + 2 * j + 1];
+          if (QT == 0) {
+            w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r),
+                              q_int8_bits(b.y, r));
+          } else {
+            w[j] = e4m3x2_bits(a.x * r, a.y * r) | (e4m3x2_bits(b.x * r, b.y * r) << 16);
+          }
+        }
+        dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_3d(&tm_q, s_out + par * out_stride, 0, 0, tile * p.nr);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait<0>();
+}
+
+// ------------------------------------------------------------------------------------------
+// rotq_cols: rotation along dimension 0.  A cluster of CTAs covers one strip
+// of 32 columns over all rows; its CTAs split the 128-row blocks of the strip.
+// Lane (p, h) of a warp owns columns (2p, 2p+1) of the strip and the 64 rows
+// of a 128-row block with row parity h; the bottom butterfly stage is formed
+// while loading (each lane reads both rows of a pair), the other six run on
+// the lane's own rows.  The column maximum needs the whole column, so the
+// strip is streamed twice: pass 1 reduces the maxima (warp -> CTA -> cluster
+// through distributed shared memory), pass 2 re-reads the strip (an L2 hit:
+// a cluster's strip is at most a few MB) and writes the codes.
+// ------------------------------------------------------------------------------------------
+struct RotqColsParams {
+  float* scales;
+  int64_t cols;
+  int nblocks;     // rows / 128
+  int warps;       // warps per CTA
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(128))
+};
+
+constexpr int kColsStrip = 32;
+constexpr int kColsInBytes = 128 * kColsStrip * 2;  // one 128 x 32 bf16 block
+constexpr int kColsOutBytes = 128 * kColsStrip;     // one 128 x 32 block of codes
+constexpr int kColsStages = 2;
+
+template <int QT>
+__global__ void __launch_bounds__(128)
+    rotq_cols_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                     RotqColsParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t bars[4][kColsStages];
+  __shared__ uint32_t s_part[kColsStrip];
+  __shared__ float s_colmax[kColsStrip];
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int pcol = lane & 15;  // column pair within the strip
+  const int h = lane >> 4;     // row parity
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const int c0 = blockIdx.y * kColsStrip;
+
+  uint8_t* s_in = smem + warp * (kColsStages * kColsInBytes);
+  uint8_t* s_out = smem + p.warps * (kColsStages * kColsInBytes) + warp * (2 * kColsOutBytes);
+
+  if (threadIdx.x < kColsStrip) s_part[threadIdx.x] = 0u;
+  if (lane == 0) {
+    for (int s = 0; s < kColsStages; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // This warp's blocks: b_i = crank + csize * (warp + warps * i).
+  const int first = static_cast<int>(crank) + static_cast<int>(csize) * warp;
+  const int step = static_cast<int>(csize) * p.warps;
+  const int nmine = first < p.nblocks ? (p.nblocks - first + step - 1) / step : 0;
+  const int nseq = 2 * nmine;  // pass 1 then pass 2 over the same blocks
+
+  auto issue = [&](int j) {
+    const int b = first + step * (j < nmine ? j : j - nmine);
+    const int s = j % kColsStages;
+    mbar_arrive_expect_tx(&bars[warp][s], kColsInBytes);
+    tma_load_2d(s_in + s * kColsInBytes, &tm_x, &bars[warp][s], c0, b * 128);
+  };
+  if (lane == 0) {
+    for (int j = 0; j < kColsStages && j < nseq; ++j) issue(j);
+  }
+
+  bool failed = false;
+  float m0 = 0.f, m1 = 0.f;   // this lane's column maxima (pass 1)
+  float r0 = 0.f, r1 = 0.f;   // quantisation multipliers (pass 2)
+
+  for (int j = 0; j < nseq; ++j) {
+    if (j == nmine) {
+      // End of pass 1 for this warp: fold the two row parities, publish to the CTA.
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
+      if (h == 0) {
+        atomicMax(&s_part[2 * pcol], __float_as_uint(m0));
+        atomicMax(&s_part[2 * pcol + 1], __float_as_uint(m1));
+      }
+      break;  // pass 2 continues after the cluster-wide reduction below
+    }
+    const int s = j % kColsStages;
+    const uint32_t ph = (j / kColsStages) & 1u;
+    const bool ok = mbar_wait(&bars[warp][s], ph, kSiteRotqColsLoad);
+    if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
+    const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
+    float2 v[64];
+    const float sg = h ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
+      const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
+      v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
+    }
+    __syncwarp();
+    if (lane == 0 && j + kColsStages < nseq) issue(j + kColsStages);
+#pragma unroll
+    for (int hp = 1; hp < 64; hp *= 2) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        if ((i & hp) == 0) {
+          const float2 a = v[i], b = v[i + hp];
+          v[i] = f2_add(a, b);
+          v[i + hp] = f2_sub(a, b);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      m0 = fmaxf(m0, fabsf(v[i].x));
+      m1 = fmaxf(m1, fabsf(v[i].y));
+    }
+  }
+  // Cluster-wide column maxima through distributed shared memory.
+  __syncthreads();
+  cluster_arrive();
+  cluster_wait();
+  if (threadIdx.x < kColsStrip) {
+    uint32_t mx = 0u;
+    for (uint32_t r = 0; r < csize; ++r) {
+      const uint32_t v = ld_shared_cluster_u32(map_to_rank(&s_part[threadIdx.x], r));
+      mx = mx > v ? mx : v;
+    }
+    const float cm = __uint_as_float(mx);
+    s_colmax[threadIdx.x] = cm;
+    const int64_t col = c0 + threadIdx.x;
+    if (crank == 0 && col < p.cols) p.scales[col] = cm * p.scale_mult;
+  }
+  __syncthreads();
+  cluster_arrive();  // this CTA no longer reads remote shared memory
+
+  {
+    const float cm0 = s_colmax[2 * pcol], cm1 = s_colmax[2 * pcol + 1];
+    r0 = cm0 > 0.f ? __fdiv_rn(p.qmax, cm0) : 0.f;
+    r1 = cm1 > 0.f ? __fdiv_rn(p.qmax, cm1) : 0.f;
+  }
+
+  for (int j = nmine; j < nseq && !failed; ++j) {
+    const int s = j % kColsStages;
+    const uint32_t ph = (j / kColsStages) & 1u;
+    const int ob = (j - nmine) & 1;
+    const bool ok = mbar_wait(&bars[warp][s], ph, kSiteRotqColsLoad);
+    if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
+    const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
+    float2 v[64];
+    const float sg = h ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
+      const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
+      v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (j + kColsStages < nseq) issue(j + kColsStages);
+      bulk_wait_read<1>();  // code buffer `ob` (used two blocks ago) is free again
+    }
+#pragma unroll
+    for (int hp = 1; hp < 64; hp *= 2) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        if ((i & hp) == 0) {
+          const float2 a = v[i], b = v[i + hp];
+          v[i] = f2_add(a, b);
+          v[i + hp] = f2_sub(a, b);
+        }
+      }
+    }
+    __syncwarp();
+    uint16_t* outw = reinterpret_cast<uint16_t*>(s_out + ob * kColsOutBytes);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      uint32_t code;
+      if (QT == 0) {
+        code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
+      } else {
+        code = e4m3x2_bits(v[i].x * r0, v[i].y * r1);
+      }
+      outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int b = first + step * (j - nmine);
+      tma_store_2d(&tm_q, s_out + ob * kColsOutBytes, c0, b * 128);
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait<0>();
+  cluster_wait();  // every CTA of the cluster is done reading this CTA's s_part
+}
+
+}  // namespace halo

@@ -1,0 +1,173 @@
+/*
+ * halo.h -- C ABI of the B200 (sm_100a) Hadamard-rotated quantized linear layer.
+ *
+ * The operation: "HALO: Hadamard-Assisted Lower-Precision Optimization for
+ * LLMs" (arXiv 2501.02625, abstract) places Hadamard rotations in the forward
+ * and backward passes of a transformer's linear layers so that every large
+ * matrix multiplication runs in low precision (INT8 or FP8: same page, "key
+ * design").  For nn.Linear shapes X[M,K], W[N,K]:
+ *     Y  = X  W^T   contraction over K      (forward)
+ *     dX = dY W     contraction over N      (backward, input gradient)
+ *     dW = dY^T X   contraction over M      (backward, weight gradient)
+ * each GEMM rotates both operands along its contraction dimension with a
+ * block-local Walsh-Hadamard transform (blocks of 128 or 256 consecutive
+ * elements, natural Sylvester order, normalised by 1/sqrt(blk): QWHA page,
+ * sec. 2.1-2.2 for the transform, HALO blog page sec. 5 for block locality),
+ * quantises each operand symmetrically with one fp32 scale per
+ * non-contraction index (scale = max|v| / qmax, q = round-half-even(v /
+ * scale), INT8 qmax 127 clamped to +-127, E4M3 qmax 448 saturating: QWHA page
+ * sec. 2.2 "quantize"), multiplies the codes on the tensor cores with int32 /
+ * fp32 accumulation, and dequantises with the product of the two scales.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates device memory; scratch comes from the caller's
+ *     workspace (see halo_workspace_size).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream; nothing is
+ *     synchronised by the library.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid argument returns an error status and launches nothing.
+ *   - Matrices are row-major with an explicit leading dimension `ld_*` counted
+ *     in ELEMENTS.  bf16 = 2 bytes, INT8 / E4M3 codes = 1 byte.
+ *   - Alignment: every pointer must be 16-byte aligned and every row stride
+ *     must be a multiple of 16 bytes (the tensor-memory-accelerator copy
+ *     rule); otherwise HALO_ERR_ALIGN.
+ *   - A device that is not compute capability 10.0 (B200 / sm_100a) gives
+ *     HALO_ERR_UNSUPPORTED.  There is no fallback path.
+ *   - Kernels bound every wait they make; a wait that runs out records a
+ *     device-side error that halo_device_error() reports (HALO_ERR_TIMEOUT).
+ */
+#ifndef HALO_H_
+#define HALO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HALO_OK = 0,
+  HALO_ERR_NULL = 1,        /* a required pointer is NULL                      */
+  HALO_ERR_SHAPE = 2,       /* a size <= 0, a dimension not a multiple of blk, */
+                            /* or a size beyond a documented limit             */
+  HALO_ERR_BLOCK = 3,       /* blk not supported for this call                 */
+  HALO_ERR_ALIGN = 4,       /* pointer not 16-byte aligned / stride rule       */
+  HALO_ERR_DTYPE = 5,       /* unknown qtype / otype / axis / major            */
+  HALO_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required         */
+  HALO_ERR_CUDA = 7,        /* a CUDA runtime / driver call failed             */
+  HALO_ERR_TIMEOUT = 8,     /* a kernel's bounded wait ran out                 */
+  HALO_ERR_UNSUPPORTED = 9  /* device is not sm_100 (B200)                     */
+} halo_status_t;
+
+typedef enum { HALO_Q_INT8 = 0, HALO_Q_E4M3 = 1 } halo_qtype_t;
+typedef enum { HALO_OUT_FP32 = 0, HALO_OUT_BF16 = 1 } halo_otype_t;
+
+/* Rotation axis of halo_hadamard_quantize. */
+typedef enum {
+  HALO_AXIS_COLS = 0, /* rotate along the contiguous dimension (blocks of blk
+                         consecutive elements of a row); one scale per ROW    */
+  HALO_AXIS_ROWS = 1  /* rotate along dimension 0 (blocks of blk consecutive
+                         rows of a column); one scale per COLUMN              */
+} halo_axis_t;
+
+/* Storage order of a GEMM operand of halo_qgemm. */
+typedef enum {
+  HALO_MAJOR_K = 0,  /* A stored [M, K] (B stored [N, K]): contraction dim contiguous */
+  HALO_MAJOR_MN = 1  /* A stored [K, M] (B stored [K, N]): the other dim contiguous   */
+} halo_major_t;
+
+/*
+ * Rotate + quantise one bf16 matrix X[rows, cols] (row stride ld_x elements).
+ *   axis = HALO_AXIS_COLS: cols % blk == 0, blk in {128, 256}, cols <= 32768.
+ *       scales_out[rows]:  s_r = max_c |Xrot[r, c]| / qmax.
+ *   axis = HALO_AXIS_ROWS: rows % blk == 0, blk == 128, cols % 8 == 0.
+ *       scales_out[cols]:  s_c = max_r |Xrot[r, c]| / qmax.
+ * Xrot is X with every block transformed by H_blk / sqrt(blk).  q_out[rows,
+ * cols] (row stride ld_q bytes) receives q = round-half-even(Xrot / s)
+ * clamped to +-127 as two's-complement int8 (qtype INT8), or Xrot / s rounded
+ * to nearest-even and saturated to +-448 as OCP E4M3 bytes (qtype E4M3).  A
+ * group whose max is 0 gets scale 0 and all-zero codes.  The codes keep the
+ * input's layout in both axes (nothing is transposed); halo_qgemm reads the
+ * dimension-0-rotated codes as an MN-major operand.
+ * Defined by: HALO paper page (abstract; "key design": INT8 or FP8); QWHA page
+ * sec. 2.1-2.2 (Walsh-Hadamard transform, symmetric quantiser).
+ */
+halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                                     int axis, int blk, int qtype, void* q_out, int64_t ld_q,
+                                     float* scales_out, void* stream);
+
+/*
+ * Low-precision GEMM on codes with a dequantising epilogue:
+ *     C[i, j] = (sum_k A[i, k] B[j, k]) * s_a[i] * s_b[j]
+ * A is M x K and B is N x K (logically).  a_major / b_major give their
+ * storage: HALO_MAJOR_K means A stored [M, K] with row stride ld_a (B: [N, K],
+ * ld_b); HALO_MAJOR_MN means A stored [K, M] (B: [K, N]) with that row stride.
+ * INT8 codes accumulate exactly in int32 (requires K * 127^2 < 2^31, i.e.
+ * K <= 133144); E4M3 codes accumulate in fp32.  C is [M, N] with row stride
+ * ld_c elements, fp32 or bf16 (round-to-nearest-even of the fp32 value).
+ * Strides: ld_a, ld_b multiples of 16; ld_c * sizeof(C element) multiple of 16.
+ * Defined by: HALO paper page, abstract ("all large matrix multiplications
+ * ... executed in lower precision") and "key design" (INT8 or FP8).
+ */
+halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a,
+                         const void* b_q, const float* s_b, int b_major, int64_t ld_b, int64_t m,
+                         int64_t n, int64_t k, int qtype, void* c, int otype, int64_t ld_c,
+                         void* stream);
+
+/*
+ * Scratch bytes halo_linear_fwd (which = 0) or halo_linear_bwd (which = 1)
+ * needs for these sizes: the operands' codes and scales.
+ */
+size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which);
+
+/*
+ * Forward linear layer Y[M, N] = X[M, K] W[N, K]^T with both operands
+ * rotated along K (blocks of blk, K % blk == 0), quantised per row (qtype),
+ * multiplied on codes and dequantised.  x, w, y dense row-major.  ws must hold
+ * halo_workspace_size(m, n, k, 0) bytes and be 16-byte aligned.
+ * Defined by: HALO paper page, abstract (rotations in the forward pass).
+ */
+halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
+                              int64_t k, int blk, int qtype, void* y, int otype, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/*
+ * Backward linear layer for Y = X W^T, given dY[M, N], X[M, K], W[N, K]:
+ *   dX[M, K] = dY W:    dY rotated along N per row, W rotated along N
+ *                       (dimension 0) per column; requires N % blk == 0.
+ *   dW[N, K] = dY^T X:  dY and X both rotated along M (dimension 0), one
+ *                       scale per column; requires M % blk == 0.
+ * blk must be 128.  dx or dw may be NULL to skip that product (the inputs it
+ * alone needs may then be NULL too).  All matrices dense row-major.  ws must
+ * hold halo_workspace_size(m, n, k, 1) bytes.
+ * Defined by: HALO paper page, abstract (rotations in the backward pass so that
+ * both backward matmuls run in low precision).
+ */
+halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const void* w_bf16,
+                              int64_t m, int64_t n, int64_t k, int blk, int qtype, void* dx,
+                              int otype_dx, void* dw, int otype_dw, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* halo_status_string(int status);
+
+/*
+ * Synchronises the current device, then reports and clears the device-side
+ * error word that kernels set when a bounded wait runs out.  Returns HALO_OK
+ * when no kernel recorded an error, HALO_ERR_TIMEOUT when one did (the kernel
+ * site is written to *where if where != NULL), HALO_ERR_CUDA when the
+ * synchronisation itself failed.
+ */
+halo_status_t halo_device_error(int* where);
+
+/* The last CUDA error code seen by the library on this thread (0 if none). */
+int halo_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HALO_H_ */

@@ -57,6 +57,9 @@ def _load():
         "halo_oracle_e4m3_decode": (D, [ctypes.c_uint8]),
         "halo_oracle_e4m3_encode": (ctypes.c_uint8, [D]),
         "halo_oracle_boundary_distance": (D, [D, I]),
+        "halo_oracle_e4m3_encode_array": (None, [P, I64, P]),
+        "halo_oracle_e4m3_decode_array": (None, [P, I64, P]),
+        "halo_oracle_boundary_distance_array": (None, [P, I64, I, P]),
         "halo_oracle_quantize": (None, [P, I64, I64, I, I, P, P, P]),
         "halo_oracle_gemm_i8": (None, [P, P, I64, I64, I64, P]),
         "halo_oracle_gemm_e4m3": (None, [P, P, I64, I64, I64, P]),
@@ -151,15 +154,17 @@ def quantize(v: np.ndarray, axis: int, qtype: int):
 
 
 def e4m3_encode(t) -> np.ndarray:
-    lib = _load()
-    flat = np.asarray(t, dtype=np.float64).ravel()
-    return np.array([lib.halo_oracle_e4m3_encode(float(v)) for v in flat], dtype=np.uint8).reshape(np.shape(t))
+    flat = np.ascontiguousarray(np.asarray(t, dtype=np.float64).ravel())
+    out = np.empty(flat.shape, dtype=np.uint8)
+    _load().halo_oracle_e4m3_encode_array(_ptr(flat), flat.size, _ptr(out))
+    return out.reshape(np.shape(t))
 
 
 def e4m3_decode(codes) -> np.ndarray:
-    lib = _load()
-    flat = np.asarray(codes, dtype=np.uint8).ravel()
-    return np.array([lib.halo_oracle_e4m3_decode(int(c)) for c in flat], dtype=np.float64).reshape(np.shape(codes))
+    flat = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8).ravel())
+    out = np.empty(flat.shape, dtype=np.float64)
+    _load().halo_oracle_e4m3_decode_array(_ptr(flat), flat.size, _ptr(out))
+    return out.reshape(np.shape(codes))
 
 
 def e4m3_decode_table() -> np.ndarray:
@@ -168,15 +173,10 @@ def e4m3_decode_table() -> np.ndarray:
 
 def boundary_distance(t: np.ndarray, qtype: int) -> np.ndarray:
     """Distance of each pre-rounding value to its nearest rounding midpoint, relative to |t|."""
-    lib = _load()
-    flat = np.asarray(t, dtype=np.float64).ravel()
-    if qtype == INT8:
-        a = np.abs(flat)
-        d = np.abs(a - (np.floor(a) + 0.5))
-        with np.errstate(divide="ignore", invalid="ignore"):
-            out = np.where(a == 0, np.inf, d / np.where(a == 0, 1, a))
-        return out.reshape(np.shape(t))
-    return np.array([lib.halo_oracle_boundary_distance(float(v), qtype) for v in flat]).reshape(np.shape(t))
+    flat = np.ascontiguousarray(np.asarray(t, dtype=np.float64).ravel())
+    out = np.empty(flat.shape, dtype=np.float64)
+    _load().halo_oracle_boundary_distance_array(_ptr(flat), flat.size, qtype, _ptr(out))
+    return out.reshape(np.shape(t))
 
 
 def gemm_i8(a: np.ndarray, b: np.ndarray) -> np.ndarray:

@@ -182,6 +182,19 @@ double halo_oracle_boundary_distance(double t, int qtype) {
   return d / a;
 }
 
+/* Array forms of the two functions above (same arithmetic, element by element). */
+void halo_oracle_e4m3_encode_array(const double* t, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = halo_oracle_e4m3_encode(t[i]);
+}
+
+void halo_oracle_e4m3_decode_array(const uint8_t* codes, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = halo_oracle_e4m3_decode(codes[i]);
+}
+
+void halo_oracle_boundary_distance_array(const double* t, int64_t n, int qtype, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = halo_oracle_boundary_distance(t[i], qtype);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Symmetric absmax quantisation (QWHA page sec. 2.2 quantize, read as      */
 /* q = round(x / (absmax / qmax))).  One scale per group; a group is a row  */

@@ -1,0 +1,128 @@
+"""The C ABI library loads, exports every symbol include/halo.h declares, and
+rejects invalid arguments on the host before touching the GPU (no CUDA call is
+made by any check in this file)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from hadamard_rotated_precision_halo_b200 import build as halo_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "halo.h")
+
+OK, NULL, SHAPE, BLOCK, ALIGN, DTYPE, WORKSPACE = 0, 1, 2, 3, 4, 5, 6
+
+FAKE = 0x100000  # a 16-byte-aligned address that is never dereferenced by these calls
+MISALIGNED = 0x100008
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = halo_build.build()
+    import hadamard_rotated_precision_halo_b200 as h
+
+    return h.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(halo_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("halo_hadamard_quantize", "halo_qgemm", "halo_linear_fwd", "halo_linear_bwd",
+                     "halo_workspace_size", "halo_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", halo_build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (halo_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_binding_covers_every_export():
+    import hadamard_rotated_precision_halo_b200 as h
+
+    assert set(h.EXPORTS) == set(declared_functions())
+
+
+def test_status_strings(lib):
+    for s in range(10):
+        assert lib.halo_status_string(s).decode().startswith("HALO")
+    assert b"unknown" in lib.halo_status_string(99)
+
+
+def test_workspace_size(lib):
+    m, n, k = 1024, 512, 768
+    fwd = lib.halo_workspace_size(m, n, k, 0)
+    assert fwd >= m * k + n * k + 4 * (m + n)
+    bwd = lib.halo_workspace_size(m, n, k, 1)
+    assert bwd >= 2 * m * n + n * k + m * k + 4 * (m + 2 * n + k)
+    assert lib.halo_workspace_size(0, n, k, 0) == 0
+    assert lib.halo_workspace_size(m, n, k, 7) == 0
+
+
+def _hq(lib, x=FAKE, rows=256, cols=512, ld_x=512, axis=0, blk=128, qt=0, q=FAKE, ld_q=512, s=FAKE):
+    return lib.halo_hadamard_quantize(x, rows, cols, ld_x, axis, blk, qt, q, ld_q, s, None)
+
+
+def test_hadamard_quantize_host_validation(lib):
+    assert _hq(lib, x=None) == NULL
+    assert _hq(lib, s=None) == NULL
+    assert _hq(lib, qt=5) == DTYPE
+    assert _hq(lib, axis=3) == DTYPE
+    assert _hq(lib, blk=64) == BLOCK
+    assert _hq(lib, axis=1, blk=256) == BLOCK
+    assert _hq(lib, cols=500, ld_x=512, ld_q=512) == SHAPE       # not a multiple of blk
+    assert _hq(lib, rows=0) == SHAPE
+    assert _hq(lib, cols=65536, ld_x=65536, ld_q=65536) == SHAPE  # beyond the row-kernel limit
+    assert _hq(lib, axis=1, rows=200) == SHAPE                    # rows % 128
+    assert _hq(lib, ld_x=256) == SHAPE                            # ld < cols
+    assert _hq(lib, x=MISALIGNED) == ALIGN
+    assert _hq(lib, ld_x=516, ld_q=516) == ALIGN                  # bf16 row stride not 16 B
+
+
+def _gemm(lib, a=FAKE, sa=FAKE, am=0, lda=256, b=FAKE, sb=FAKE, bm=0, ldb=256, m=128, n=128, k=256, qt=0,
+          c=FAKE, ot=0, ldc=128):
+    return lib.halo_qgemm(a, sa, am, lda, b, sb, bm, ldb, m, n, k, qt, c, ot, ldc, None)
+
+
+def test_qgemm_host_validation(lib):
+    assert _gemm(lib, a=None) == NULL
+    assert _gemm(lib, c=None) == NULL
+    assert _gemm(lib, qt=2) == DTYPE
+    assert _gemm(lib, ot=2) == DTYPE
+    assert _gemm(lib, am=2) == DTYPE
+    assert _gemm(lib, m=0) == SHAPE
+    assert _gemm(lib, k=200000, lda=200000, ldb=200000) == SHAPE  # int32 accumulator bound
+    assert _gemm(lib, lda=128) == SHAPE
+    assert _gemm(lib, lda=264, ldb=264) == ALIGN
+    assert _gemm(lib, b=MISALIGNED) == ALIGN
+    assert _gemm(lib, ot=1, n=100, ldc=100) == ALIGN  # 200-byte bf16 rows
+
+
+def test_linear_host_validation(lib):
+    ws = lib.halo_workspace_size(256, 256, 512, 0)
+    f = lib.halo_linear_fwd
+    assert f(None, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, ws, None) == NULL
+    assert f(FAKE, FAKE, 256, 256, 512, 64, 0, FAKE, 0, FAKE, ws, None) == BLOCK
+    assert f(FAKE, FAKE, 256, 256, 500, 128, 0, FAKE, 0, FAKE, ws, None) == SHAPE
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, None, ws, None) == WORKSPACE
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, ws - 1, None) == WORKSPACE
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 9, FAKE, 0, FAKE, ws, None) == DTYPE
+    wsb = lib.halo_workspace_size(256, 256, 512, 1)
+    b = lib.halo_linear_bwd
+    assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, None, 0, None, 0, FAKE, wsb, None) == NULL
+    assert b(FAKE, None, FAKE, 256, 256, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == NULL  # dW needs X
+    assert b(FAKE, FAKE, FAKE, 256, 256, 512, 256, 0, FAKE, 0, FAKE, 0, FAKE, wsb, None) == BLOCK
+    assert b(FAKE, FAKE, FAKE, 200, 256, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == SHAPE  # M % 128
+    assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE

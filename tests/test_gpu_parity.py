@@ -1,0 +1,251 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on seeded inputs.
+
+Small cases span several tiles and ragged tails and are compared element by
+element; the full Llama-shaped cases run in the benchmark's launch
+configuration and are compared on sampled rows / columns that the oracle
+computes one by one (each row or column of a rotated-quantised operand depends
+on that row or column alone).
+"""
+import numpy as np
+import pytest
+import torch
+
+import hadamard_rotated_precision_halo_b200 as halo
+import oracle
+from hadamard_rotated_precision_halo_b200 import inputs
+from tests._parity import OUT_REL, check_codes, check_output, oracle_operand, u8
+
+pytestmark = pytest.mark.gpu
+
+INT8, E4M3 = halo.HALO_Q_INT8, halo.HALO_Q_E4M3
+FP32, BF16 = halo.HALO_OUT_FP32, halo.HALO_OUT_BF16
+COLS, ROWS = halo.HALO_AXIS_COLS, halo.HALO_AXIS_ROWS
+
+
+@pytest.fixture(autouse=True)
+def no_device_error():
+    yield
+    st, site = halo.halo_device_error()
+    assert st == halo.HALO_OK, f"kernel bounded wait ran out at site {site:#x}"
+
+
+def _cuda(t):
+    return t.to("cuda")
+
+
+# ------------------------------------------------------------------ rotate + quantise
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols,blk", [(300, 640, 128), (130, 512, 256), (1, 128, 128), (64, 256, 256),
+                                           (37, 11008, 128), (5, 28672, 128)])
+def test_rotq_rows_parity(qtype, rows, cols, blk):
+    x = inputs.activations(rows, cols, seed=rows * 7 + cols, device="cpu")
+    x[min(3, rows - 1)] = 0  # an all-zero row: scale 0, codes 0
+    q, s = halo.halo_hadamard_quantize(_cuda(x), COLS, blk, qtype)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle_operand(x, 1, blk, qtype)
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols", [(1024, 208), (384, 96), (2048, 64), (128, 16), (4096, 48)])
+def test_rotq_cols_parity(qtype, rows, cols):
+    x = inputs.activations(rows, cols, seed=rows + 3 * cols, device="cpu")
+    x[:, min(5, cols - 1)] = 0  # an all-zero column
+    q, s = halo.halo_hadamard_quantize(_cuda(x), ROWS, 128, qtype)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle_operand(x, 0, 128, qtype)
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+def test_rotq_rows_strided_input():
+    base = inputs.activations(96, 768, seed=11, device="cpu")
+    x = base[:, :512]  # row stride 768 elements
+    xd = _cuda(base)[:, :512]
+    q, s = halo.halo_hadamard_quantize(xd, COLS, 128, INT8)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle_operand(x.contiguous(), 1, 128, INT8)
+    check_codes(q, s, codes, scales, t, INT8)
+
+
+# ------------------------------------------------------------------------------ GEMM
+def _rand_codes(rows, cols, qtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    if qtype == INT8:
+        return torch.randint(-127, 128, (rows, cols), generator=g, dtype=torch.int8)
+    b = torch.randint(0, 256, (rows, cols), generator=g, dtype=torch.int16).to(torch.uint8)
+    b[(b & 0x7F) == 0x7F] = 0x38  # no NaN codes
+    return b.view(torch.float8_e4m3fn)
+
+
+def _stored(codes_logical: torch.Tensor, major: int) -> torch.Tensor:
+    """Storage of a logical [rows, K] operand: K-major as is, MN-major transposed."""
+    return codes_logical if major == halo.HALO_MAJOR_K else codes_logical.t().contiguous()
+
+
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1), (0, 1), (1, 0)])
+@pytest.mark.parametrize("m,n,k", [(300, 520, 640), (128, 256, 128), (16, 16, 208), (640, 272, 1024)])
+def test_qgemm_int8_bit_exact(a_major, b_major, m, n, k):
+    if a_major == 1 and m % 16 or b_major == 1 and n % 16:
+        pytest.skip("MN-major storage needs a 16-byte row stride")
+    a = _rand_codes(m, k, INT8, seed=m + k)
+    b = _rand_codes(n, k, INT8, seed=n * 3 + k)
+    ones_m = torch.ones(m, dtype=torch.float32, device="cuda")
+    ones_n = torch.ones(n, dtype=torch.float32, device="cuda")
+    c = halo.halo_qgemm(_cuda(_stored(a, a_major)), ones_m, a_major, _cuda(_stored(b, b_major)), ones_n, b_major,
+                        m, n, k, INT8, FP32)
+    torch.cuda.synchronize()
+    acc = oracle.gemm_i8(a.numpy(), b.numpy())
+    # with unit scales the output is exactly float32(acc): bit-exact int32 accumulation
+    np.testing.assert_array_equal(c.cpu().numpy(), acc.astype(np.float32))
+
+
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1)])
+@pytest.mark.parametrize("otype", [FP32, BF16])
+def test_qgemm_e4m3_with_scales(a_major, b_major, otype):
+    m, n, k = 272, 528, 768
+    a = _rand_codes(m, k, E4M3, seed=5)
+    b = _rand_codes(n, k, E4M3, seed=6)
+    g = torch.Generator().manual_seed(7)
+    sa = torch.rand(m, generator=g) + 0.5
+    sb = torch.rand(n, generator=g) * 1e-3 + 1e-4
+    c = halo.halo_qgemm(_cuda(_stored(a, a_major)), _cuda(sa), a_major, _cuda(_stored(b, b_major)), _cuda(sb),
+                        b_major, m, n, k, E4M3, otype)
+    torch.cuda.synchronize()
+    ref = oracle.dequant(oracle.gemm_e4m3(a.view(torch.uint8).numpy(), b.view(torch.uint8).numpy()), sa.numpy(),
+                         sb.numpy())
+    err = check_output(c, ref)
+    if otype == FP32:
+        assert err < 1e-5  # fp32 accumulation of exact E4M3 products
+
+
+def test_qgemm_int8_scales_epilogue():
+    m, n, k = 256, 512, 512
+    a = _rand_codes(m, k, INT8, seed=1)
+    b = _rand_codes(n, k, INT8, seed=2)
+    g = torch.Generator().manual_seed(3)
+    sa = torch.rand(m, generator=g) * 0.01
+    sb = torch.rand(n, generator=g) * 0.01
+    c = halo.halo_qgemm(_cuda(a), _cuda(sa), 0, _cuda(b), _cuda(sb), 0, m, n, k, INT8, FP32)
+    torch.cuda.synchronize()
+    ref = oracle.dequant(oracle.gemm_i8(a.numpy(), b.numpy()).astype(np.float64), sa.numpy(), sb.numpy())
+    err = check_output(c, ref)
+    assert err < 1e-6
+
+
+# ---------------------------------------------------------------------- linear layer
+def test_linear_fwd_tiny_config():
+    """X[64,256], W[128,256] ~ N(0,1), seed 0; one 256-block on K; INT8; Y fp32."""
+    x = inputs.plain(64, 256, seed=0, device="cpu")
+    w = inputs.plain(128, 256, seed=1, device="cpu")
+    y = halo.halo_linear_fwd(_cuda(x), _cuda(w), 256, INT8, FP32)
+    qx, sx = halo.halo_hadamard_quantize(_cuda(x), COLS, 256, INT8)
+    qw, sw = halo.halo_hadamard_quantize(_cuda(w), COLS, 256, INT8)
+    torch.cuda.synchronize()
+    cx, osx, tx = oracle_operand(x, 1, 256, INT8)
+    cw, osw, tw = oracle_operand(w, 1, 256, INT8)
+    check_codes(qx, sx, cx, osx, tx, INT8)
+    check_codes(qw, sw, cw, osw, tw, INT8)
+    ref = oracle.linear_fwd(x, w, 256, INT8)
+    check_output(y, ref)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("otype", [FP32, BF16])
+def test_linear_fwd_parity(qtype, otype):
+    m, n, k = 384, 320, 640
+    x = inputs.activations(m, k, seed=21, device="cpu")
+    w = inputs.weights(n, k, seed=22, device="cpu")
+    y = halo.halo_linear_fwd(_cuda(x), _cuda(w), 128, qtype, otype)
+    torch.cuda.synchronize()
+    check_output(y, oracle.linear_fwd(x, w, 128, qtype))
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+def test_linear_bwd_parity(qtype):
+    m, n, k = 512, 384, 640
+    dy = inputs.grads(m, n, seed=31, device="cpu")
+    x = inputs.activations(m, k, seed=32, device="cpu")
+    w = inputs.weights(n, k, seed=33, device="cpu")
+    dx, dw = halo.halo_linear_bwd(_cuda(dy), _cuda(x), _cuda(w), 128, qtype, BF16, FP32)
+    torch.cuda.synchronize()
+    check_output(dx, oracle.linear_bwd_dx(dy, w, 128, qtype))
+    check_output(dw, oracle.linear_bwd_dw(dy, x, 128, qtype))
+
+
+def test_linear_bwd_single_products():
+    m, n, k = 256, 256, 384
+    dy = inputs.grads(m, n, seed=41, device="cpu")
+    x = inputs.activations(m, k, seed=42, device="cpu")
+    w = inputs.weights(n, k, seed=43, device="cpu")
+    dx, _ = halo.halo_linear_bwd(_cuda(dy), None, _cuda(w), 128, INT8, FP32, FP32, want_dw=False)
+    _, dw = halo.halo_linear_bwd(_cuda(dy), _cuda(x), None, 128, INT8, FP32, FP32, want_dx=False)
+    torch.cuda.synchronize()
+    check_output(dx, oracle.linear_bwd_dx(dy, w, 128, INT8))
+    check_output(dw, oracle.linear_bwd_dw(dy, x, 128, INT8))
+
+
+# --------------------------------------------------------------- full Llama-shaped cases
+def _sampled_gemm_ref(a_rows_bf16, a_along, b_rows_bf16, b_along, blk, qtype):
+    """Oracle values C[i, j] for a sample of A's and B's logical rows.
+
+    a_rows_bf16: the sampled part of A's storage -- rows of A when a_along == 1
+    (rotate along its contiguous dim), columns of A^T's storage (as a [K, r]
+    matrix) when a_along == 0.  Same for B."""
+    ca, sa, _ = oracle_operand(a_rows_bf16, a_along, blk, qtype)
+    cb, sb, _ = oracle_operand(b_rows_bf16, b_along, blk, qtype)
+    if a_along == 0:
+        ca = np.ascontiguousarray(ca.T)
+    if b_along == 0:
+        cb = np.ascontiguousarray(cb.T)
+    acc = oracle.gemm_i8(ca, cb).astype(np.float64) if qtype == INT8 else oracle.gemm_e4m3(ca, cb)
+    return oracle.dequant(acc, sa, sb)
+
+
+def _sample(n, count, seed):
+    g = np.random.default_rng(seed)
+    idx = np.sort(g.choice(n, size=min(count, n), replace=False))
+    idx[-1] = n - 1  # always include the last (ragged-tail) index
+    return idx
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+def test_full_rotate_quantize_16384x4096(qtype):
+    x = inputs.activations(16384, 4096, seed=1, device="cuda")
+    q, s = halo.halo_hadamard_quantize(x, COLS, 128, qtype)
+    torch.cuda.synchronize()
+    rows = _sample(16384, 256, 1)
+    xs = x[torch.from_numpy(rows).cuda()].cpu()
+    codes, scales, t = oracle_operand(xs, 1, 128, qtype)
+    check_codes(q[torch.from_numpy(rows).cuda()], s[torch.from_numpy(rows).cuda()], codes, scales, t, qtype)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+def test_full_forward_8192x4096x4096(qtype):
+    m, n, k = 8192, 4096, 4096
+    x = inputs.activations(m, k, seed=2, device="cuda")
+    w = inputs.weights(n, k, seed=3, device="cuda")
+    y = halo.halo_linear_fwd(x, w, 128, qtype, BF16)
+    torch.cuda.synchronize()
+    ri, ci = _sample(m, 48, 4), _sample(n, 64, 5)
+    ref = _sampled_gemm_ref(x[torch.from_numpy(ri).cuda()].cpu(), 1, w[torch.from_numpy(ci).cuda()].cpu(), 1, 128,
+                            qtype)
+    check_output(y[torch.from_numpy(ri).cuda()][:, torch.from_numpy(ci).cuda()], ref)
+
+
+def test_full_backward_8192x11008x4096():
+    m, n, k = 8192, 4096, 11008
+    dy = inputs.grads(m, n, seed=5, device="cuda")
+    w = inputs.weights(n, k, seed=6, device="cuda")
+    x = inputs.activations(m, k, seed=7, device="cuda")
+    dx, dw = halo.halo_linear_bwd(dy, x, w, 128, INT8, BF16, FP32)
+    torch.cuda.synchronize()
+    # dX[M, K] = dY W: A rows = dY rows (rotated along N), B rows = W columns (rotated along dim 0 of W)
+    ri, ci = _sample(m, 32, 8), _sample(k, 48, 9)
+    ri_t, ci_t = torch.from_numpy(ri).cuda(), torch.from_numpy(ci).cuda()
+    ref = _sampled_gemm_ref(dy[ri_t].cpu(), 1, w[:, ci_t].cpu(), 0, 128, INT8)
+    check_output(dx[ri_t][:, ci_t], ref)
+    # dW[N, K] = dY^T X: A rows = dY columns, B rows = X columns, both rotated along M
+    ni, ki = _sample(n, 32, 10), _sample(k, 48, 11)
+    ni_t, ki_t = torch.from_numpy(ni).cuda(), torch.from_numpy(ki).cuda()
+    ref = _sampled_gemm_ref(dy[:, ni_t].cpu(), 0, x[:, ki_t].cpu(), 0, 128, INT8)
+    check_output(dw[ni_t][:, ki_t], ref)
