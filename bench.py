@@ -257,31 +257,51 @@ def e2e_run(step: LayerStep, steps: int):
 
 
 # ------------------------------------------------------------------ CPU baseline
-def cpu_baseline(seconds_target: float = 15.0):
-    """The oracle as it stands, on a bounded sample of the layer step: the q
-    projection forward (rotate + quantise X rows and all of W_q, integer GEMM,
-    dequantise) restricted to the first R token rows."""
-    import oracle
+class OracleSample:
+    """The oracle as it stands on a bounded sample of the layer step: the q
+    projection forward (rotate + quantise the first `rows` token rows of X and
+    all of W_q, integer GEMM, dequantise)."""
 
-    shapes = inputs.LLAMA70B_LAYER
-    g = shapes.gemms[0]
-    oracle.build()
-    w = inputs.weights(g.n, g.k, seed=100, device="cpu")
-    rows = 16
-    x = inputs.activations(rows, g.k, seed=101, device="cpu")
-    t0 = time.perf_counter()
-    oracle.linear_fwd(x, w, BLK, oracle.INT8)
-    dt = time.perf_counter() - t0
-    if dt < seconds_target / 3:
-        rows = int(min(512, rows * max(1.0, seconds_target / max(dt, 1e-3) * 0.8)))
-        x = inputs.activations(rows, g.k, seed=101, device="cpu")
+    def __init__(self):
+        import oracle
+
+        self.oracle = oracle
+        oracle.build()
+        self.g = inputs.LLAMA70B_LAYER.gemms[0]
+        self.w = inputs.weights(self.g.n, self.g.k, seed=100, device="cpu")
+        self.x_all = inputs.activations(inputs.LLAMA70B_LAYER.tokens, self.g.k, seed=101, device="cpu")
+        self.rows = 16
+
+    def run(self, rows=None):
+        rows = rows or self.rows
+        x = self.x_all[:rows]
         t0 = time.perf_counter()
-        oracle.linear_fwd(x, w, BLK, oracle.INT8)
+        self.oracle.linear_fwd(x, self.w, BLK, self.oracle.INT8)
         dt = time.perf_counter() - t0
-    ops = 2 * rows * g.n * g.k
-    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"q-projection forward, {rows} of {shapes.tokens} token rows x W[{g.n},{g.k}], "
-                      f"INT8, block 128 ({dt:.1f} s)"}
+        return 2 * rows * self.g.n * self.g.k, dt
+
+    def size_for(self, seconds: float):
+        """Grow the row sample until one run takes about `seconds`."""
+        rows = 16
+        ops, dt = self.run(rows)
+        cap = self.x_all.shape[0]
+        while dt < 0.6 * seconds and rows < cap:
+            rows = min(cap, rows * 2)
+            ops, dt = self.run(rows)
+        self.rows = rows
+        return ops, dt
+
+    def describe(self, dt):
+        return (f"q-projection forward, {self.rows} of {inputs.LLAMA70B_LAYER.tokens} token rows x "
+                f"W[{self.g.n},{self.g.k}] (rotate+quantise both, INT8 GEMM, dequantise), block 128, "
+                f"{dt:.1f} s per sample")
+
+
+def cpu_baseline(seconds_target: float = 15.0):
+    s = OracleSample()
+    ops, dt = s.size_for(seconds_target)
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": s.oracle.num_threads(), "kind": "oracle",
+            "sample": s.describe(dt)}
 
 
 # ------------------------------------------------------------------------- main
@@ -307,12 +327,23 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        cb = cpu_baseline()
-        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
-                "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        s = OracleSample()
+        s.size_for(4.0)
+        for _ in range(args.warmup):
+            s.run()
+        ops_total, t_total = 0, 0.0
+        for _ in range(args.steps):
+            ops, dt = s.run()
+            ops_total += ops
+            t_total += dt
+        value = ops_total / t_total / 1e12
+        cb = {"value": value, "unit": UNIT, "cores": s.oracle.num_threads(), "kind": "oracle",
+              "sample": s.describe(t_total / max(args.steps, 1))}
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(args.steps, 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config, "cpu_baseline": cb,
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
 

@@ -46,6 +46,7 @@ EXPORTS = (
     "halo_status_string",
     "halo_device_error",
     "halo_last_cuda_error",
+    "halo_last_error_detail",
 )
 
 _lib = None
@@ -56,7 +57,7 @@ class HaloError(RuntimeError):
         self.status = status
         msg = status_text(status)
         if status == HALO_ERR_CUDA and _lib is not None:
-            msg += f" (cuda error {_lib.halo_last_cuda_error()})"
+            msg += f" (cuda error {_lib.halo_last_cuda_error()}: {_lib.halo_last_error_detail().decode()})"
         super().__init__(f"{what}: {msg}" if what else msg)
 
 
@@ -88,6 +89,8 @@ def lib():
     L.halo_device_error.restype = I
     L.halo_last_cuda_error.argtypes = []
     L.halo_last_cuda_error.restype = I
+    L.halo_last_error_detail.argtypes = []
+    L.halo_last_error_detail.restype = ctypes.c_char_p
     _lib = L
     return L
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
@@ -18,6 +19,7 @@ using namespace halo;
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+thread_local char g_last_detail[256] = "";
 
 constexpr int kMaxDevices = 64;
 
@@ -34,20 +36,27 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-halo_status_t cuda_fail(cudaError_t e) {
+halo_status_t cuda_fail(cudaError_t e, const char* what) {
   g_last_cuda_error = static_cast<int>(e);
+  snprintf(g_last_detail, sizeof g_last_detail, "%s: %s", what, cudaGetErrorString(e));
   return HALO_ERR_CUDA;
 }
 
-#define HALO_CUDA(call)                         \
-  do {                                          \
-    cudaError_t e_ = (call);                    \
-    if (e_ != cudaSuccess) return cuda_fail(e_); \
+#define HALO_CUDA(call)                                  \
+  do {                                                   \
+    cudaError_t e_ = (call);                             \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);  \
   } while (0)
 
+// Let a kernel use all the dynamic shared memory it may: the opt-in limit
+// minus its static shared memory.
 template <typename K>
-cudaError_t set_smem_attr(K kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+cudaError_t set_smem_attr(K kernel, int optin) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
@@ -71,18 +80,22 @@ halo_status_t device_setup(int* dev_out) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
       HALO_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
-      if (q != cudaDriverEntryPointSuccess || !fn) return HALO_ERR_CUDA;
+      if (q != cudaDriverEntryPointSuccess || !fn) {
+        snprintf(g_last_detail, sizeof g_last_detail, "cuTensorMapEncodeTiled entry point not found");
+        return HALO_ERR_CUDA;
+      }
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
-    const size_t big = 227 * 1024;
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 0>, big));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 1>, big));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 0>, big));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 1>, big));
-    HALO_CUDA(set_smem_attr(rotq_cols_kernel<0>, big));
-    HALO_CUDA(set_smem_attr(rotq_cols_kernel<1>, big));
-    HALO_CUDA(set_smem_attr(qgemm_kernel<0>, kGemmSmemBytes));
-    HALO_CUDA(set_smem_attr(qgemm_kernel<1>, kGemmSmemBytes));
+    int optin = 0;
+    HALO_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 0>, optin));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 1>, optin));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 0>, optin));
+    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 1>, optin));
+    HALO_CUDA(set_smem_attr(rotq_cols_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(rotq_cols_kernel<1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_kernel<1>, optin));
   }
   d.ready = true;
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
@@ -97,7 +110,11 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    g_last_cuda_error = static_cast<int>(r);
+    g_last_cuda_error = 10000 + static_cast<int>(r);
+    snprintf(g_last_detail, sizeof g_last_detail,
+             "cuTensorMapEncodeTiled(rank %d, dims %llu x %llu, box %u x %u) failed with CUresult %d", rank,
+             static_cast<unsigned long long>(dims[0]), static_cast<unsigned long long>(dims[1]), box[0], box[1],
+             static_cast<int>(r));
     return HALO_ERR_CUDA;
   }
   return HALO_OK;
@@ -384,6 +401,8 @@ const char* halo_status_string(int status) {
 }
 
 int halo_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* halo_last_error_detail(void) { return g_last_detail; }
 
 halo_status_t halo_device_error(int* where) {
   HALO_CUDA(cudaDeviceSynchronize());

@@ -163,8 +163,13 @@ const char* halo_status_string(int status);
  */
 halo_status_t halo_device_error(int* where);
 
-/* The last CUDA error code seen by the library on this thread (0 if none). */
+/* The last CUDA error code seen by the library on this thread (0 if none).
+ * A failed tensor-map encoding is reported as 10000 + its CUresult. */
 int halo_last_cuda_error(void);
+
+/* Text naming the last failing CUDA call on this thread ("" if none).  The
+ * string is owned by the library and stays valid until the next failure. */
+const char* halo_last_error_detail(void);
 
 #ifdef __cplusplus
 }

@@ -38,18 +38,26 @@ def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype):
     return int(exempt.sum()), int((diff & exempt).sum())
 
 
+def bf16_half_ulp(y: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers (8 significant bits) at |y|."""
+    a = np.abs(y)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 8), 0.0)
+
+
 def check_output(gpu_out: torch.Tensor, ref: np.ndarray, rel: float = OUT_REL):
+    """max |Y - Y_ref| / max |Y_ref| <= rel.  For bf16 outputs the bound applies to
+    the value before the final rounding, so each element may differ by a further
+    half bf16 ulp of itself (the rounding to bf16 alone is up to 2^-9 relative)."""
     y = gpu_out.detach().float().cpu().numpy().astype(np.float64)
     assert y.shape == ref.shape
     assert np.all(np.isfinite(y))
     scale = np.max(np.abs(ref))
-    err = np.max(np.abs(y - ref)) / (scale if scale > 0 else 1.0)
-    assert err <= rel, f"normwise error {err:.3e} > {rel:.1e}"
+    diff = np.abs(y - ref)
     if gpu_out.dtype == torch.bfloat16:
-        # beyond the normwise bound, most elements sit within one bf16 ulp
-        big = np.abs(ref) > 1e-2 * scale
-        r = np.abs(y[big] - ref[big]) / np.abs(ref[big])
-        assert np.median(r) <= 2.0**-8
+        diff = np.maximum(diff - bf16_half_ulp(y), 0.0)
+    err = np.max(diff) / (scale if scale > 0 else 1.0)
+    assert err <= rel, f"normwise error {err:.3e} > {rel:.1e}"
     return err
 
 
