@@ -43,6 +43,7 @@ EXPORTS = (
     "halo_workspace_size",
     "halo_linear_fwd",
     "halo_linear_bwd",
+    "halo_linear_fwd_noalloc",
     "halo_status_string",
     "halo_device_error",
     "halo_last_cuda_error",
@@ -83,6 +84,8 @@ def lib():
     L.halo_linear_fwd.restype = I
     L.halo_linear_bwd.argtypes = [P, P, P, I64, I64, I64, I, I, P, I, P, I, P, SZ, P]
     L.halo_linear_bwd.restype = I
+    L.halo_linear_fwd_noalloc.argtypes = [P, P, I64, I64, I64, I, I, P, I, P]
+    L.halo_linear_fwd_noalloc.restype = I
     L.halo_status_string.argtypes = [I]
     L.halo_status_string.restype = ctypes.c_char_p
     L.halo_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]

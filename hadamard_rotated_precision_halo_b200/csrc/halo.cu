@@ -16,6 +16,12 @@
 
 using namespace halo;
 
+// Scratch of halo_linear_fwd_noalloc: codes and scales of X and W live here
+// instead of in a caller workspace.  Host code must not use this name as an
+// address (it is a host-side stand-in); the device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HALO_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 thread_local int g_last_cuda_error = 0;
@@ -99,6 +105,20 @@ halo_status_t device_setup(int* dev_out) {
   }
   d.ready = true;
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+}
+
+// Device address of g_noalloc_scratch, one per device, set on the first
+// halo_linear_fwd_noalloc call made with that device current.
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+halo_status_t noalloc_setup(int dev) {
+  if (g_noalloc_ptr[dev]) return HALO_OK;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_noalloc_ptr[dev]) return HALO_OK;
+  void* p = nullptr;
+  HALO_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+  g_noalloc_ptr[dev] = p;
+  return HALO_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -464,6 +484,29 @@ halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m,
   if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_COLS, blk, qtype, xq, k, sx, stream)) != HALO_OK) return st;
   if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_COLS, blk, qtype, wq, k, sw, stream)) != HALO_OK) return st;
   return halo_qgemm(xq, sx, HALO_MAJOR_K, k, wq, sw, HALO_MAJOR_K, k, m, n, k, qtype, y, otype, n, stream);
+}
+
+halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k,
+                                      int blk, int qtype, void* y, int otype, void* stream) {
+  // Argument checks of halo_linear_fwd and the scratch limit come first, so
+  // that nothing touches the device on input this call would reject.
+  if (!x_bf16 || !w_bf16 || !y) return HALO_ERR_NULL;
+  if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
+  if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
+  if (m <= 0 || n <= 0 || k <= 0 || k % blk != 0 || k > 32768) return HALO_ERR_SHAPE;
+  const size_t need = ws_layout(m, n, k, 0).total;
+  if (need > HALO_NOALLOC_SCRATCH_BYTES) {
+    snprintf(g_last_detail, sizeof g_last_detail,
+             "halo_linear_fwd_noalloc: these sizes need %zu bytes of scratch, the library's static array holds %llu",
+             need, static_cast<unsigned long long>(HALO_NOALLOC_SCRATCH_BYTES));
+    return HALO_ERR_WORKSPACE;
+  }
+  int dev = 0;
+  halo_status_t st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  if ((st = noalloc_setup(dev)) != HALO_OK) return st;
+  return halo_linear_fwd(x_bf16, w_bf16, m, n, k, blk, qtype, y, otype, g_noalloc_ptr[dev],
+                         HALO_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,

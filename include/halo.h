@@ -151,6 +151,43 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
                               int otype_dx, void* dw, int otype_dw, void* ws, size_t ws_bytes,
                               void* stream);
 
+/*
+ * Size of the library-owned scratch array used by halo_linear_fwd_noalloc.
+ */
+#define HALO_NOALLOC_SCRATCH_BYTES (64ull << 20) /* 64 MiB */
+
+/*
+ * Forward linear layer computed exactly as halo_linear_fwd, but for callers
+ * that cannot allocate device memory.  There is no counterpart in the paper:
+ * this is an interface variant, not part of the method.
+ *
+ * Who needs it: code that only ever receives input and output pointers and has
+ * no way to obtain scratch -- for example a plugin inside an inference server
+ * or framework whose interface hands over no workspace, or a latency-critical
+ * loop that must not call cudaMalloc, because cudaMalloc can synchronise the
+ * device and stall every other stream.  Such a caller passes X, W and Y only.
+ *
+ * Where the scratch comes from: a file-scope __device__ array of
+ * HALO_NOALLOC_SCRATCH_BYTES inside the library.  Every GPU that loads the
+ * library holds that array until the process exits.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Limits and behaviour:
+ *   - Arguments and layout as for halo_linear_fwd.  Sizes whose codes and
+ *     scales do not fit (halo_workspace_size(m, n, k, 0) greater than
+ *     HALO_NOALLOC_SCRATCH_BYTES) return HALO_ERR_WORKSPACE and launch nothing;
+ *     halo_last_error_detail() then gives the bytes needed.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Nothing in it has to start at zero: a call reads only bytes it wrote
+ *     earlier in the same call.  Calls that can overlap on the GPU (on
+ *     unordered streams, or from several host threads) race on the array;
+ *     order them on one stream or with events.
+ */
+halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
+                                      int64_t k, int blk, int qtype, void* y, int otype, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* halo_status_string(int status);
 

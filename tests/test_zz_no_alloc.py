@@ -1,0 +1,64 @@
+"""halo_linear_fwd_noalloc: the forward linear layer for callers that cannot
+allocate device memory (for instance a plugin whose host interface hands it
+only input and output pointers, or a loop that must not call cudaMalloc
+because it can synchronise the device).  Its scratch is a fixed array inside
+the library, so the call takes X, W and Y only.
+
+This file is collected last on purpose.  Its test must give the same result as
+the workspace entry point, on two calls in a row (the shared array keeps the
+previous call's contents), both in a fresh process and after every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import hadamard_rotated_precision_halo_b200 as halo
+from hadamard_rotated_precision_halo_b200 import inputs
+from tests._parity import check_output
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 64 << 20  # HALO_NOALLOC_SCRATCH_BYTES in include/halo.h
+
+
+def _call(lib, x, w, y, blk, qtype, otype):
+    m, k = x.shape
+    n = w.shape[0]
+    return lib.halo_linear_fwd_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()), m, n, k, blk,
+                                       qtype, ctypes.c_void_p(y.data_ptr()), otype,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("qtype,otype", [(halo.HALO_Q_INT8, halo.HALO_OUT_FP32),
+                                         (halo.HALO_Q_E4M3, halo.HALO_OUT_BF16)])
+def test_noalloc_forward_matches_workspace_forward(qtype, otype):
+    lib = halo.lib()
+    m, n, k, blk = 1024, 768, 2048, 128
+    assert lib.halo_workspace_size(m, n, k, 0) <= SCRATCH_BYTES
+    x = inputs.activations(m, k, seed=61, device="cuda")
+    w = inputs.weights(n, k, seed=62, device="cuda")
+    ref = halo.halo_linear_fwd(x, w, blk, qtype, otype)  # the existing entry point, caller workspace
+    torch.cuda.synchronize()
+    ref_np = ref.float().cpu().numpy().astype(np.float64)
+    out_dtype = torch.float32 if otype == halo.HALO_OUT_FP32 else torch.bfloat16
+    for _ in range(2):  # the second call finds the first call's codes still in the array
+        y = torch.full((m, n), float("nan"), dtype=out_dtype, device="cuda")
+        st = _call(lib, x, w, y, blk, qtype, otype)
+        assert st == halo.HALO_OK, halo.status_text(st)
+        torch.cuda.synchronize()
+        check_output(y, ref_np)
+    st, site = halo.halo_device_error()
+    assert st == halo.HALO_OK, f"bounded wait ran out at site {site:#x}"
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    lib = halo.lib()
+    m, n, k = 8192, 8192, 4096  # 64 MiB of codes alone, plus scales
+    assert lib.halo_workspace_size(m, n, k, 0) > SCRATCH_BYTES
+    x = torch.empty((16, 16), dtype=torch.bfloat16, device="cuda")  # never read: rejected before any launch
+    st = lib.halo_linear_fwd_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(x.data_ptr()), m, n, k, 128,
+                                     halo.HALO_Q_INT8, ctypes.c_void_p(x.data_ptr()), halo.HALO_OUT_FP32, None)
+    assert st == halo.HALO_ERR_WORKSPACE
+    assert b"scratch" in lib.halo_last_error_detail()
