@@ -108,10 +108,11 @@ class ClockSampler:
 class LayerStep:
     """All tensors and launches of one layer step (forward + dX + dW of 7 GEMMs)."""
 
-    def __init__(self, shapes: inputs.LayerShapes, seed: int, device, qtype: int):
+    def __init__(self, shapes: inputs.LayerShapes, seed: int, device, qtype: int, kinds=("fwd", "dx", "dw")):
         import hadamard_rotated_precision_halo_b200 as halo
 
         self.halo = halo
+        self.kinds = kinds
         self.shapes = shapes
         self.qtype = qtype
         self.dev = device
@@ -138,7 +139,7 @@ class LayerStep:
         self.ws = torch.empty(max(self.ws_fwd, self.ws_bwd), dtype=torch.uint8, device=device)
 
     def ops_per_step(self) -> int:
-        return self.shapes.total_ops()
+        return self.shapes.total_ops(self.kinds)
 
     def _codes(self, buf, rows, cols):
         return buf[: rows * cols].view(self.code_dt).view(rows, cols)
@@ -150,11 +151,14 @@ class LayerStep:
         out = []
         for g in self.shapes.gemms:
             x, w = self.t["x"][g.x_key], self.t["w"][g.name]
-            out.append(("fwd", g.name, x, h.HALO_AXIS_COLS, w, h.HALO_AXIS_COLS, t, g.n, g.k, self.y[g.name]))
+            if "fwd" in self.kinds:
+                out.append(("fwd", g.name, x, h.HALO_AXIS_COLS, w, h.HALO_AXIS_COLS, t, g.n, g.k, self.y[g.name]))
         for g in self.shapes.gemms:
             x, w, dy = self.t["x"][g.x_key], self.t["w"][g.name], self.t["dy"][g.name]
-            out.append(("dx", g.name, dy, h.HALO_AXIS_COLS, w, h.HALO_AXIS_ROWS, t, g.k, g.n, self.dx[g.name]))
-            out.append(("dw", g.name, dy, h.HALO_AXIS_ROWS, x, h.HALO_AXIS_ROWS, g.n, g.k, t, self.dw[g.name]))
+            if "dx" in self.kinds:
+                out.append(("dx", g.name, dy, h.HALO_AXIS_COLS, w, h.HALO_AXIS_ROWS, t, g.k, g.n, self.dx[g.name]))
+            if "dw" in self.kinds:
+                out.append(("dw", g.name, dy, h.HALO_AXIS_ROWS, x, h.HALO_AXIS_ROWS, g.n, g.k, t, self.dw[g.name]))
         return out
 
     def run(self, events=None):
@@ -177,6 +181,10 @@ class LayerStep:
             st = L.halo_hadamard_quantize(h._ptr(a), a.shape[0], a.shape[1], a.stride(0), a_axis, BLK, self.qtype,
                                           h._ptr(qa), qa.stride(0), h._ptr(self.sa), sp)
             h._check(st, "rotq A")
+            if events is not None:
+                events["mid"].append(torch.cuda.Event(enable_timing=True))
+                events["mid"][-1].record(stream)
+                events["axes"].append((a_axis, b_axis, a.numel(), b.numel()))
             st = L.halo_hadamard_quantize(h._ptr(b), b.shape[0], b.shape[1], b.stride(0), b_axis, BLK, self.qtype,
                                           h._ptr(qb), qb.stride(0), h._ptr(self.sb), sp)
             h._check(st, "rotq B")
@@ -305,6 +313,13 @@ def cpu_baseline(seconds_target: float = 15.0):
 
 
 # ------------------------------------------------------------------------- main
+WORKLOADS = {
+    "llama70b_layer_fwd_bwd": (inputs.LLAMA70B_LAYER, ("fwd", "dx", "dw")),
+    "llama7b_attn_proj_fwd": (inputs.LLAMA7B_ATTN_PROJ, ("fwd",)),
+    "llama7b_ffn_down_bwd": (inputs.LLAMA7B_FFN_DOWN, ("dx", "dw")),
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -314,15 +329,17 @@ def main():
     ap.add_argument("--qtype", default="int8", choices=["int8", "e4m3"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="llama70b_layer_fwd_bwd", choices=sorted(WORKLOADS),
+                    help="the bench line uses the default; the single-GEMM cases serve profiling")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    shapes = inputs.LLAMA70B_LAYER
-    config = {"workload": "llama70b_layer_fwd_bwd", "tokens": shapes.tokens, "hidden": shapes.hidden,
-              "ffn": shapes.ffn, "kv": shapes.kv, "gemms": 21, "block": BLK, "qtype": args.qtype,
-              "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
+    shapes, kinds = WORKLOADS[args.workload]
+    config = {"workload": args.workload, "tokens": shapes.tokens, "hidden": shapes.hidden,
+              "ffn": shapes.ffn, "kv": shapes.kv, "gemms": len(shapes.gemms) * len(kinds), "block": BLK,
+              "qtype": args.qtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -356,7 +373,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     qtype = halo.HALO_Q_INT8 if args.qtype == "int8" else halo.HALO_Q_E4M3
-    step = LayerStep(shapes, seed=4 + rank, device=device, qtype=qtype)
+    step = LayerStep(shapes, seed=4 + rank, device=device, qtype=qtype, kinds=kinds)
     torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
@@ -366,7 +383,7 @@ def main():
     if st != halo.HALO_OK:
         raise RuntimeError(f"device error after warm-up at site {site:#x}")
 
-    events = {"rotq": [], "gemm": [], "end": []}
+    events = {"rotq": [], "mid": [], "gemm": [], "end": [], "axes": []}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -391,6 +408,13 @@ def main():
         raise RuntimeError(f"device error in the timed region at site {site:#x}")
 
     rotq_ms = sum(a.elapsed_time(b) for a, b in zip(events["rotq"], events["gemm"]))
+    # per rotation direction: [ms, elements] for axis COLS (rotq_rows kernel) and ROWS (rotq_cols kernels)
+    by_axis = {0: [0.0, 0], 1: [0.0, 0]}
+    for e0, e1, e2, (ax_a, ax_b, na, nb) in zip(events["rotq"], events["mid"], events["gemm"], events["axes"]):
+        by_axis[ax_a][0] += e0.elapsed_time(e1)
+        by_axis[ax_a][1] += na
+        by_axis[ax_b][0] += e1.elapsed_time(e2)
+        by_axis[ax_b][1] += nb
     gemm_ms = sum(a.elapsed_time(b) for a, b in zip(events["gemm"], events["end"]))
     n_gemm = len(events["gemm"])
     ops_step = step.ops_per_step()
@@ -413,7 +437,11 @@ def main():
                          "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']})",
                          "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
             "rotq": {"gbs": rotq_gbs, "peak_gbs": pk["hbm_gbs"], "frac": rotq_gbs / pk["hbm_gbs"],
-                     "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps},
+                     "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps,
+                     "along_contiguous_dim_gbs": 3 * by_axis[0][1] / (by_axis[0][0] * 1e-3) / 1e9,
+                     "along_dim0_gbs": 3 * by_axis[1][1] / (by_axis[1][0] * 1e-3) / 1e9,
+                     "along_contiguous_dim_ms_per_step": by_axis[0][0] / args.steps,
+                     "along_dim0_ms_per_step": by_axis[1][0] / args.steps},
             "clocks": clocks.summary()}
 
     if rank == 0 and not args.no_e2e:

@@ -65,6 +65,22 @@ cudaError_t set_smem_attr(K kernel, int optin) {
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
+typedef void (*Cols1Kernel)(const CUtensorMap, const CUtensorMap, RotqCols1Params);
+
+template <int QT>
+Cols1Kernel cols_1pass_for(int nw) {
+  switch (nw) {
+    case 1: return rotq_cols_1pass_kernel<QT, 1>;
+    case 2: return rotq_cols_1pass_kernel<QT, 2>;
+    case 3: return rotq_cols_1pass_kernel<QT, 3>;
+    default: return rotq_cols_1pass_kernel<QT, 4>;
+  }
+}
+
+Cols1Kernel cols_1pass_kernel(int qtype, int nw) {
+  return qtype == HALO_Q_INT8 ? cols_1pass_for<0>(nw) : cols_1pass_for<1>(nw);
+}
+
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
 // driver entry point for tensor-map encoding.
 halo_status_t device_setup(int* dev_out) {
@@ -100,6 +116,12 @@ halo_status_t device_setup(int* dev_out) {
     HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 1>, optin));
     HALO_CUDA(set_smem_attr(rotq_cols_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(rotq_cols_kernel<1>, optin));
+    for (int nw = 1; nw <= 4; ++nw) {
+      for (int qt = 0; qt < 2; ++qt) {
+        HALO_CUDA(set_smem_attr(cols_1pass_kernel(qt, nw), optin));
+        HALO_CUDA(cudaFuncSetAttribute(cols_1pass_kernel(qt, nw), cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+      }
+    }
     HALO_CUDA(set_smem_attr(qgemm_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_kernel<1>, optin));
   }
@@ -195,9 +217,67 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   return HALO_OK;
 }
 
+// Single pass when the 128-row blocks of a column strip split evenly over a
+// cluster of at most 16 CTAs with at most 4 warps each (R <= 8192 rows).
+halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
+                                     int64_t ld_q, float* scales, cudaStream_t stream, int nw, int cl, int dev) {
+  const int strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  RotqCols1Params p;
+  p.scales = scales;
+  p.cols = cols;
+  p.strips = strips;
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  Cols1Kernel kern = cols_1pass_kernel(qtype, nw);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(32 * nw, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(nw) * (2 * kColsInBytes + kColsOutBytes) + 128;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Persistent: as many clusters as fit at once (each loops over strips).
+  cfg.gridDim = dim3(cl, 1, 1);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1) {
+    (void)cudaGetLastError();
+    max_clusters = std::max(1, g_dev[dev].sm_count / cl);
+  }
+  cfg.gridDim = dim3(cl, std::min(strips, max_clusters), 1);
+  HALO_CUDA(cudaLaunchKernelEx(&cfg, kern, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
 halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
-                               int64_t ld_q, float* scales, cudaStream_t stream) {
+                               int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
   const int nblocks = static_cast<int>(rows / 128);
+  for (int nw = 4; nw >= 1; --nw) {
+    if (nblocks % nw == 0 && nblocks / nw <= 16)
+      return launch_rotq_cols_1pass(x, rows, cols, ld_x, qtype, q, ld_q, scales, stream, nw, nblocks / nw, dev);
+  }
+  // Taller matrices: the two-pass kernel (column maxima first, then codes).
   int cl = 8;
   while (cl > 1 && cl > nblocks) cl /= 2;
   const int warps = std::max(1, std::min(4, (nblocks + cl - 1) / cl));
@@ -448,7 +528,7 @@ halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t c
   if (st != HALO_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (axis == HALO_AXIS_COLS) return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, qtype, q_out, ld_q, scales_out, s, dev);
-  return launch_rotq_cols(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, s);
+  return launch_rotq_cols(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, s, dev);
 }
 
 halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,

@@ -182,6 +182,58 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return r;
 }
 
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Remote atomic max on a cluster peer's shared memory (relaxed, cluster scope).
+__device__ __forceinline__ void red_max_shared_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.max.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Arrive on a cluster peer's mbarrier, releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a local mbarrier whose arrivals come from cluster peers
+// (acquire at cluster scope, so their prior writes are visible afterwards).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t phase, unsigned int site) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, phase)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(a, phase)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      record_error(site);
+      return false;
+    }
+  }
+}
+
+// 16-byte store into a cluster peer's shared memory that completes 16 bytes
+// of transaction count on the peer's mbarrier `bar` (both peer addresses).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");

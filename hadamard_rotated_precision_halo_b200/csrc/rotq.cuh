@@ -255,6 +255,57 @@ __global__ void __launch_bounds__(256, 1)
 // through distributed shared memory), pass 2 re-reads the strip (an L2 hit:
 // a cluster's strip is at most a few MB) and writes the codes.
 // ------------------------------------------------------------------------------------------
+constexpr int kColsStrip = 32;
+constexpr int kColsInBytes = 128 * kColsStrip * 2;  // one 128 x 32 bf16 block
+constexpr int kColsOutBytes = 128 * kColsStrip;     // one 128 x 32 block of codes
+constexpr int kColsStages = 2;
+
+// Lane (pcol, h) of a warp owns columns (2 pcol, 2 pcol + 1) and the 64 rows
+// 2i + h of a 128-row block held in shared memory as [128][32] bf16.  Reading
+// both rows of every pair forms the bottom butterfly stage on the way in
+// (h = 0 keeps the sum, h = 1 the difference); the other six stages run on
+// the lane's own rows.
+__device__ __forceinline__ void cols_load_fwht(const uint32_t* blkw, int pcol, int h, float2 (&v)[64]) {
+  const float sg = h ? -1.f : 1.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
+    const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
+    v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
+  }
+}
+
+__device__ __forceinline__ void cols_fwht_rest(float2 (&v)[64]) {
+#pragma unroll
+  for (int hp = 1; hp < 64; hp *= 2) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      if ((i & hp) == 0) {
+        const float2 a = v[i], b = v[i + hp];
+        v[i] = f2_add(a, b);
+        v[i + hp] = f2_sub(a, b);
+      }
+    }
+  }
+}
+
+// Codes of the lane's 64 rows x 2 columns into a [128][32]-byte tile.
+template <int QT>
+__device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
+                                                 int h) {
+  uint16_t* outw = reinterpret_cast<uint16_t*>(tile);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    uint32_t code;
+    if (QT == 0) {
+      code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
+    } else {
+      code = e4m3x2_bits(v[i].x * r0, v[i].y * r1);
+    }
+    outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
+  }
+}
+
 struct RotqColsParams {
   float* scales;
   int64_t cols;
@@ -263,11 +314,6 @@ struct RotqColsParams {
   float qmax;
   float scale_mult;  // 1 / (qmax * sqrt(128))
 };
-
-constexpr int kColsStrip = 32;
-constexpr int kColsInBytes = 128 * kColsStrip * 2;  // one 128 x 32 bf16 block
-constexpr int kColsOutBytes = 128 * kColsStrip;     // one 128 x 32 block of codes
-constexpr int kColsStages = 2;
 
 template <int QT>
 __global__ void __launch_bounds__(128)
@@ -334,26 +380,10 @@ __global__ void __launch_bounds__(128)
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
-    const float sg = h ? -1.f : 1.f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
-      const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
-      v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
-    }
+    cols_load_fwht(blkw, pcol, h, v);
     __syncwarp();
     if (lane == 0 && j + kColsStages < nseq) issue(j + kColsStages);
-#pragma unroll
-    for (int hp = 1; hp < 64; hp *= 2) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        if ((i & hp) == 0) {
-          const float2 a = v[i], b = v[i + hp];
-          v[i] = f2_add(a, b);
-          v[i + hp] = f2_sub(a, b);
-        }
-      }
-    }
+    cols_fwht_rest(v);
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
       m0 = fmaxf(m0, fabsf(v[i].x));
@@ -392,41 +422,15 @@ __global__ void __launch_bounds__(128)
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
-    const float sg = h ? -1.f : 1.f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
-      const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
-      v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
-    }
+    cols_load_fwht(blkw, pcol, h, v);
     __syncwarp();
     if (lane == 0) {
       if (j + kColsStages < nseq) issue(j + kColsStages);
       bulk_wait_read<1>();  // code buffer `ob` (used two blocks ago) is free again
     }
-#pragma unroll
-    for (int hp = 1; hp < 64; hp *= 2) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        if ((i & hp) == 0) {
-          const float2 a = v[i], b = v[i + hp];
-          v[i] = f2_add(a, b);
-          v[i + hp] = f2_sub(a, b);
-        }
-      }
-    }
+    cols_fwht_rest(v);
     __syncwarp();
-    uint16_t* outw = reinterpret_cast<uint16_t*>(s_out + ob * kColsOutBytes);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      uint32_t code;
-      if (QT == 0) {
-        code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
-      } else {
-        code = e4m3x2_bits(v[i].x * r0, v[i].y * r1);
-      }
-      outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
-    }
+    cols_write_codes<QT>(s_out + ob * kColsOutBytes, v, r0, r1, pcol, h);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -437,6 +441,161 @@ __global__ void __launch_bounds__(128)
   }
   if (lane == 0) bulk_wait<0>();
   cluster_wait();  // every CTA of the cluster is done reading this CTA's s_part
+}
+
+
+// ------------------------------------------------------------------------------------------
+// rotq_cols_1pass: rotation along dimension 0 when a 32-column strip's
+// 128-row blocks split over a cluster of at most 16 CTAs of NW <= 4 warps, one
+// block per warp (R = CL * NW * 128 <= 8192 rows).  Every rotated value stays
+// in registers while the column maxima are reduced, so the input is read once
+// and the codes written once.
+//
+// Column-max reduction per strip: warps -> CTA with shared-memory atomics and
+// one CTA barrier; then the CTA's 32 partial maxima (128 bytes) go to every
+// cluster CTA's slot [rank] with 16-byte st.async stores that complete bytes
+// on that CTA's mbarrier; each CTA waits on its own mbarrier for CL * 128
+// bytes and takes the max over the CL slots.  No cluster barrier or memory
+// fence in the loop.  Two slot buffers alternate over strips: a peer writes
+// strip k+2 only after every CTA has sent strip k+1, which each CTA does only
+// after it has read strip k.  The cluster is persistent over strips; each warp
+// prefetches its block of the next two strips with TMA.
+// ------------------------------------------------------------------------------------------
+struct RotqCols1Params {
+  float* scales;
+  int64_t cols;
+  int strips;  // ceil(cols / 32)
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(128))
+};
+
+enum : unsigned int { kSiteRotqCols1Load = 0x202, kSiteRotqCols1Reduce = 0x203 };
+
+template <int QT, int NW>
+__global__ void __launch_bounds__(NW * 32)
+    rotq_cols_1pass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                           RotqCols1Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t bars[NW][2];                            // TMA loads, per warp and stage
+  __shared__ uint64_t red_bar[2];                             // partial vectors received, per buffer
+  __shared__ uint32_t s_red[2][kColsStrip];                   // this CTA's column maxima (fp32 bits)
+  __shared__ __align__(16) uint32_t s_slot[2][16][kColsStrip];  // every cluster CTA's maxima
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int pcol = lane & 15;
+  const int h = lane >> 4;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const int blk = static_cast<int>(crank) * NW + warp;  // this warp's 128-row block
+  const uint32_t slot_bytes = csize * kColsStrip * 4;
+
+  uint8_t* s_in = smem + warp * (2 * kColsInBytes);
+  uint8_t* s_out = smem + NW * (2 * kColsInBytes) + warp * kColsOutBytes;
+
+  if (threadIdx.x < 2 * kColsStrip) (&s_red[0][0])[threadIdx.x] = 0u;
+  if (lane == 0) {
+    mbar_init(&bars[warp][0], 1);
+    mbar_init(&bars[warp][1], 1);
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&red_bar[0], 1);
+    mbar_init(&red_bar[1], 1);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&red_bar[0], slot_bytes);  // armed for strips 0 and 1
+    mbar_arrive_expect_tx(&red_bar[1], slot_bytes);
+  }
+  cluster_arrive();  // every peer is running and initialised before the first remote store
+  cluster_wait();
+
+  const int first = blockIdx.y;
+  const int step = gridDim.y;
+  const int nmine = first < p.strips ? (p.strips - first + step - 1) / step : 0;
+
+  auto issue = [&](int k) {
+    const int st = k & 1;
+    mbar_arrive_expect_tx(&bars[warp][st], kColsInBytes);
+    tma_load_2d(s_in + st * kColsInBytes, &tm_x, &bars[warp][st], (first + k * step) * kColsStrip, blk * 128);
+  };
+  if (lane == 0) {
+    if (nmine > 0) issue(0);
+    if (nmine > 1) issue(1);
+  }
+
+  bool dead = false;  // a wait ran out: stop waiting, still send every partial
+  for (int k = 0; k < nmine; ++k) {
+    const int c0 = (first + k * step) * kColsStrip;
+    const int par = k & 1;
+    float2 v[64];
+    if (!dead) {
+      const bool ok = mbar_wait(&bars[warp][par], (k >> 1) & 1, kSiteRotqCols1Load);
+      dead = __any_sync(0xffffffffu, !ok);
+    }
+    if (!dead) {
+      cols_load_fwht(reinterpret_cast<const uint32_t*>(s_in + par * kColsInBytes), pcol, h, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
+    }
+    __syncwarp();
+    if (lane == 0 && !dead && k + 2 < nmine) issue(k + 2);
+    cols_fwht_rest(v);
+    float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      m0 = fmaxf(m0, fabsf(v[i].x));
+      m1 = fmaxf(m1, fabsf(v[i].y));
+    }
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
+    if (h == 0) {
+      atomicMax(&s_red[par][2 * pcol], __float_as_uint(m0));
+      atomicMax(&s_red[par][2 * pcol + 1], __float_as_uint(m1));
+    }
+    __syncthreads();
+    if (threadIdx.x < kColsStrip / 4) {
+      // 4 columns per thread, 16 bytes to every cluster CTA's slot [crank].
+      uint4 vec = *reinterpret_cast<const uint4*>(&s_red[par][4 * threadIdx.x]);
+      *reinterpret_cast<uint4*>(&s_red[par][4 * threadIdx.x]) = make_uint4(0u, 0u, 0u, 0u);  // for strip k + 2
+      for (uint32_t r = 0; r < csize; ++r)
+        st_async_v4(map_to_rank(&s_slot[par][crank][4 * threadIdx.x], r), vec, map_to_rank(&red_bar[par], r));
+    }
+    if (!dead) {
+      const bool ok = mbar_wait_cluster(&red_bar[par], (k >> 1) & 1, kSiteRotqCols1Reduce);
+      dead = __any_sync(0xffffffffu, !ok);
+    }
+    uint32_t u0 = 0u, u1 = 0u;
+    for (uint32_t r = 0; r < csize; ++r) {
+      const uint2 pr = *reinterpret_cast<const uint2*>(&s_slot[par][r][2 * pcol]);
+      u0 = max(u0, pr.x);
+      u1 = max(u1, pr.y);
+    }
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&red_bar[par], slot_bytes);  // re-armed for strip k + 2
+    const float cm0 = __uint_as_float(u0), cm1 = __uint_as_float(u1);
+    const float r0 = cm0 > 0.f ? __fdiv_rn(p.qmax, cm0) : 0.f;
+    const float r1 = cm1 > 0.f ? __fdiv_rn(p.qmax, cm1) : 0.f;
+    if (crank == 0 && warp == 0 && h == 0) {
+      if (c0 + 2 * pcol < p.cols) p.scales[c0 + 2 * pcol] = cm0 * p.scale_mult;
+      if (c0 + 2 * pcol + 1 < p.cols) p.scales[c0 + 2 * pcol + 1] = cm1 * p.scale_mult;
+    }
+    if (lane == 0) bulk_wait_read<0>();  // the previous strip's store has read the code tile
+    __syncwarp();
+    cols_write_codes<QT>(s_out, v, r0, r1, pcol, h);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&tm_q, s_out, c0, blk * 128);
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait<0>();
+  __syncthreads();
+  cluster_arrive();  // no CTA leaves while a peer could still store into its shared memory
+  cluster_wait();
 }
 
 }  // namespace halo

@@ -82,6 +82,8 @@ class LayerShapes:
     gemms: list = field(default_factory=list)
 
     def __post_init__(self):
+        if self.gemms:
+            return  # an explicit GEMM list (a single-GEMM case)
         t, h, f, kv = self.tokens, self.hidden, self.ffn, self.kv
         self.gemms = [
             Gemm("q", t, h, h, "attn_in"),
@@ -93,12 +95,20 @@ class LayerShapes:
             Gemm("down", t, h, f, "mlp_act"),
         ]
 
-    def total_ops(self) -> int:
-        """Integer multiply-adds x2 over forward, dX and dW of all seven GEMMs."""
-        return sum(3 * 2 * g.m * g.n * g.k for g in self.gemms)
+    def total_ops(self, kinds=("fwd", "dx", "dw")) -> int:
+        """2 * M * N * K summed over the GEMMs of the listed kinds (forward, dX, dW
+        each multiply the same three sizes)."""
+        return sum(len(kinds) * 2 * g.m * g.n * g.k for g in self.gemms)
 
 
 LLAMA70B_LAYER = LayerShapes()
+# Single-GEMM Llama-7B cases: the attention projection forward (X[8192,4096],
+# W[4096,4096]) and the FFN down-projection backward (dY[8192,4096],
+# W[4096,11008], X[8192,11008]).
+LLAMA7B_ATTN_PROJ = LayerShapes(tokens=8192, hidden=4096, ffn=11008, kv=4096,
+                                gemms=[Gemm("proj", 8192, 4096, 4096, "attn_in")])
+LLAMA7B_FFN_DOWN = LayerShapes(tokens=8192, hidden=4096, ffn=11008, kv=4096,
+                               gemms=[Gemm("down", 8192, 4096, 11008, "mlp_act")])
 
 
 def layer_inputs(shapes: LayerShapes, seed: int, device) -> dict:

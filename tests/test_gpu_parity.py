@@ -47,7 +47,8 @@ def test_rotq_rows_parity(qtype, rows, cols, blk):
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
-@pytest.mark.parametrize("rows,cols", [(1024, 208), (384, 96), (2048, 64), (128, 16), (4096, 48)])
+@pytest.mark.parametrize("rows,cols", [(1024, 208), (384, 96), (2048, 64), (128, 16), (4096, 48), (1152, 48),
+                                       (8320, 32), (28672, 64)])
 def test_rotq_cols_parity(qtype, rows, cols):
     x = inputs.activations(rows, cols, seed=rows + 3 * cols, device="cpu")
     x[:, min(5, cols - 1)] = 0  # an all-zero column
