@@ -438,8 +438,8 @@ def main():
                          "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
             "rotq": {"gbs": rotq_gbs, "peak_gbs": pk["hbm_gbs"], "frac": rotq_gbs / pk["hbm_gbs"],
                      "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps,
-                     "along_contiguous_dim_gbs": 3 * by_axis[0][1] / (by_axis[0][0] * 1e-3) / 1e9,
-                     "along_dim0_gbs": 3 * by_axis[1][1] / (by_axis[1][0] * 1e-3) / 1e9,
+                     "along_contiguous_dim_gbs": 3 * by_axis[0][1] / max(by_axis[0][0] * 1e-3, 1e-12) / 1e9,
+                     "along_dim0_gbs": 3 * by_axis[1][1] / max(by_axis[1][0] * 1e-3, 1e-12) / 1e9,
                      "along_contiguous_dim_ms_per_step": by_axis[0][0] / args.steps,
                      "along_dim0_ms_per_step": by_axis[1][0] / args.steps},
             "clocks": clocks.summary()}

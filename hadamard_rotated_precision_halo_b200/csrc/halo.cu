@@ -124,6 +124,8 @@ halo_status_t device_setup(int* dev_out) {
     }
     HALO_CUDA(set_smem_attr(qgemm_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_kernel<1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1>, optin));
   }
   d.ready = true;
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
@@ -360,17 +362,20 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
       dims[0] = static_cast<cuuint64_t>(k);
       dims[1] = static_cast<cuuint64_t>(n);
       box[0] = 128;
-      box[1] = 256;
+      box[1] = m > 128 ? 128 : 256;  // the pair kernel loads 128 N indices per CTA
     }
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_b)};
     halo_status_t st = encode(&tm_b, dt, 2, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != HALO_OK) return st;
   }
+  // 256 x 256 tiles on SM pairs unless M is too small to fill a pair.
+  const bool use_pair = m > 128;
   GemmParams p;
   p.m = static_cast<int>(m);
   p.n = static_cast<int>(n);
   p.k = static_cast<int>(k);
-  p.tiles_m = static_cast<int>((m + kGemmBM - 1) / kGemmBM);
+  const int bm = use_pair ? 256 : kGemmBM;
+  p.tiles_m = static_cast<int>((m + bm - 1) / bm);
   p.tiles_n = static_cast<int>((n + kGemmBN - 1) / kGemmBN);
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.a_mn = a_mn;
@@ -385,19 +390,39 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
   idesc |= static_cast<uint32_t>(a_mn) << 15;
   idesc |= static_cast<uint32_t>(b_mn) << 16;
   idesc |= static_cast<uint32_t>(kGemmBN >> 3) << 17;
-  idesc |= static_cast<uint32_t>(kGemmBM >> 4) << 24;
+  idesc |= static_cast<uint32_t>(bm >> 4) << 24;  // M of one MMA: 128 per CTA, 256 per pair
   p.idesc = idesc;
   p.sa = sa;
   p.sb = sb;
   p.c = c;
   p.ldc = ld_c;
   p.out_bf16 = otype == HALO_OUT_BF16;
-  const int grid = std::min(p.num_tiles, g_dev[dev].sm_count);
+  if (!use_pair) {
+    const int grid = std::min(p.num_tiles, g_dev[dev].sm_count);
+    if (qtype == HALO_Q_INT8)
+      qgemm_kernel<0><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+    else
+      qgemm_kernel<1><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+    HALO_CUDA(cudaGetLastError());
+    return HALO_OK;
+  }
+  const int pairs = std::min(p.num_tiles, g_dev[dev].sm_count / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (qtype == HALO_Q_INT8)
-    qgemm_kernel<0><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+    HALO_CUDA(cudaLaunchKernelEx(&cfg, qgemm_pair_kernel<0>, tm_a, tm_b, p));
   else
-    qgemm_kernel<1><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
-  HALO_CUDA(cudaGetLastError());
+    HALO_CUDA(cudaLaunchKernelEx(&cfg, qgemm_pair_kernel<1>, tm_a, tm_b, p));
   return HALO_OK;
 }
 

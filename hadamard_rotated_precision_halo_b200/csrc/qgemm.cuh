@@ -255,4 +255,223 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+
+// ------------------------------------------------------------------------------------------
+// qgemm_pair_kernel: the same GEMM with 256 x 256 output tiles computed by a
+// pair of CTAs (a 2-CTA cluster on two SMs) with tcgen05.mma.cta_group::2.
+// Each CTA holds half of the A tile (128 rows) and half of the B tile (128
+// of the 256 N indices) in its own shared memory, so per K block an SM loads
+// 32 KB instead of 48 KB for the same tensor work.  The even CTA issues the
+// MMAs; both CTAs' TMA loads complete on the even CTA's stage barrier; the
+// MMA commits arrive on both CTAs' barriers; each CTA drains its own 128 rows
+// of the accumulator from its tensor memory and releases it on the even CTA's
+// barrier.  Loads are plain (no multicast).
+// ------------------------------------------------------------------------------------------
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = 128 * kGemmBK;  // 16 KB: 128 rows of A
+constexpr int kPairBBytes = 128 * kGemmBK;  // 16 KB: 128 N indices of B
+constexpr size_t kPairSmemBytes = kPairStages * (kPairABytes + kPairBBytes) + 1024 + 256;
+
+enum : unsigned int {
+  kSitePairProducer = 0x311,
+  kSitePairMma = 0x312,
+  kSitePairMmaAcc = 0x313,
+  kSitePairEpilogue = 0x314,
+};
+
+template <int QT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    qgemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                      GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // four epilogue warps in each CTA of the pair
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kGemmTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive();  // both CTAs' barriers and tensor memory are ready
+  cluster_wait();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kblocks = (p.k + kGemmBK - 1) / kGemmBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+        int tm, tn;
+        gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+        const int a_row = tm * 256 + static_cast<int>(rank) * 128;
+        const int b_row = tn * 256 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, kSitePairProducer)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
+          const uint32_t bar = map_to_rank(&full[stage], 0);
+          uint8_t* a_dst = sA + stage * kPairABytes;
+          uint8_t* b_dst = sB + stage * kPairBBytes;
+          if (p.a_mn)
+            tma_load_2d_pair(a_dst, &tm_a, bar, a_row, kb * kGemmBK);
+          else
+            tma_load_2d_pair(a_dst, &tm_a, bar, kb * kGemmBK, a_row);
+          if (p.b_mn)
+            tma_load_2d_pair(b_dst, &tm_b, bar, b_row, kb * kGemmBK);
+          else
+            tma_load_2d_pair(b_dst, &tm_b, bar, kb * kGemmBK, b_row);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int lt = 0;
+      const uint32_t a_step = p.a_mn ? 32u * 128u : 32u;
+      const uint32_t b_step = p.b_mn ? 32u * 128u : 32u;
+      const uint32_t lbo = p.a_mn || p.b_mn ? static_cast<uint32_t>(kGemmBK * 128) : 16u;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++lt) {
+        const uint32_t acc = lt & 1;
+        const uint32_t acc_phase = (lt >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kSitePairMmaAcc)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256u;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, kSitePairMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * kPairABytes);
+          const uint32_t b_base = smem_u32(sB + stage * kPairBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 32; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a_base + kk * a_step, p.a_mn ? lbo : 16u, 1024u);
+            const uint64_t bdesc = smem_desc_sw128(b_base + kk * b_step, p.b_mn ? lbo : 16u, 1024u);
+            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            if (QT == 0)
+              mma_i8_pair(d_tmem, adesc, bdesc, p.idesc, accumulate);
+            else
+              mma_f8_pair(d_tmem, adesc, bdesc, p.idesc, accumulate);
+          }
+          mma_commit_pair_mc(&empty[stage], 0x3);  // both CTAs' stage is free once these MMAs have read it
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        mma_commit_pair_mc(&tfull[acc], 0x3);  // both halves of the accumulator complete
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
+    const uint32_t tempty_leader1 = map_to_rank(&tempty[1], 0);
+    int lt = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++lt) {
+      int tm, tn;
+      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+      const uint32_t acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, kSitePairEpilogue);
+      if (bar_or(1, 128, !ok)) break;
+      tc_fence_after();
+      const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
+      const bool row_ok = row < p.m;
+      const float sa = row_ok ? p.sa[row] : 0.f;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256u;
+#pragma unroll 1
+      for (int ch = 0; ch < 256 / 32; ++ch) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row + ch * 32, r);
+        tmem_ld_wait();
+        const int col0 = tn * 256 + ch * 32;
+        if (row_ok && col0 < p.n) {
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = (QT == 0) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+            const int col = col0 + j;
+            const float sb = col < p.n ? __ldg(p.sb + col) : 0.f;
+            y[j] = (a * sa) * sb;
+          }
+          const bool full_chunk = col0 + 32 <= p.n;
+          if (p.out_bf16) {
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
+            if (full_chunk) {
+              uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[8 * q + 2 * e], y[8 * q + 2 * e + 1]);
+                  w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                o4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.n) out[j] = __float2bfloat16_rn(y[j]);
+            }
+          } else {
+            float* out = static_cast<float*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
+            if (full_chunk) {
+              float4* o4 = reinterpret_cast<float4*>(out);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) o4[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.n) out[j] = y[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive();  // neither CTA leaves while the other may still address its memory
+  cluster_wait();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kGemmTmemCols);
+  }
+}
+
 }  // namespace halo
