@@ -161,62 +161,114 @@ class LayerStep:
                 out.append(("dw", g.name, dy, h.HALO_AXIS_ROWS, x, h.HALO_AXIS_ROWS, g.n, g.k, t, self.dw[g.name]))
         return out
 
+    def plan(self):
+        """The step's launches in order.  An operand rotated along the same axis
+        for several GEMMs (the attention input for q, k, v and the MLP input for
+        gate, up, in the forward and in dW) is rotated once per step into a code
+        buffer of its own and reused; every other operand goes through the two
+        scratch code buffers.  Entries: ("rotq", x, axis, codes, scales) and
+        ("gemm", (codes_a, scales_a, axis_a), (codes_b, scales_b, axis_b), m, n, k, out)."""
+        if getattr(self, "_plan", None) is not None:
+            return self._plan
+        h = self.halo
+        gem = self.gemms()
+        count = {}
+        for g in gem:
+            for x, ax in ((g[2], g[3]), (g[4], g[5])):
+                key = (x.data_ptr(), ax)
+                count[key] = count.get(key, 0) + 1
+        self.shared = {}
+        for g in gem:
+            for x, ax in ((g[2], g[3]), (g[4], g[5])):
+                key = (x.data_ptr(), ax)
+                if count[key] > 1 and key not in self.shared:
+                    groups = x.shape[0] if ax == h.HALO_AXIS_COLS else x.shape[1]
+                    q = torch.empty(x.shape, dtype=self.code_dt, device=self.dev)
+                    sc = torch.empty(groups, dtype=torch.float32, device=self.dev)
+                    self.shared[key] = (q, sc)
+        plan, done = [], set()
+        for kind, name, a, a_axis, b, b_axis, m, n, k, c in gem:
+            operands = []
+            for slot, x, ax in ((0, a, a_axis), (1, b, b_axis)):
+                key = (x.data_ptr(), ax)
+                if key in self.shared:
+                    q, sc = self.shared[key]
+                    if key not in done:
+                        plan.append(("rotq", x, ax, q, sc))
+                        done.add(key)
+                else:
+                    q = self._codes(self.qa if slot == 0 else self.qb, x.shape[0], x.shape[1])
+                    sc = self.sa if slot == 0 else self.sb
+                    plan.append(("rotq", x, ax, q, sc))
+                operands.append((q, sc, ax))
+            plan.append(("gemm", operands[0], operands[1], m, n, k, c))
+        self._plan = plan
+        return plan
+
     def run(self, events=None):
-        """One step through the C ABI: per GEMM, rotate+quantise both operands
-        (halo_hadamard_quantize) and multiply (halo_qgemm).  With `events`,
-        record CUDA events around every launch (same stream)."""
+        """One step through the C ABI (halo_hadamard_quantize, halo_qgemm).  With
+        `events` (a list), record a CUDA event before every launch and one after
+        the last, on the launching stream; returns the number of launches."""
         h = self.halo
         L = h.lib()
         stream = torch.cuda.current_stream()
         sp = h._stream(stream)
-        launches = 0
-        for kind, name, a, a_axis, b, b_axis, m, n, k, c in self.gemms():
-            qa = self._codes(self.qa, a.shape[0], a.shape[1])
-            qb = self._codes(self.qb, b.shape[0], b.shape[1])
-            sa_len = a.shape[0] if a_axis == h.HALO_AXIS_COLS else a.shape[1]
-            sb_len = b.shape[0] if b_axis == h.HALO_AXIS_COLS else b.shape[1]
+        plan = self.plan()
+        for op in plan:
             if events is not None:
-                events["rotq"].append(torch.cuda.Event(enable_timing=True))
-                events["rotq"][-1].record(stream)
-            st = L.halo_hadamard_quantize(h._ptr(a), a.shape[0], a.shape[1], a.stride(0), a_axis, BLK, self.qtype,
-                                          h._ptr(qa), qa.stride(0), h._ptr(self.sa), sp)
-            h._check(st, "rotq A")
-            if events is not None:
-                events["mid"].append(torch.cuda.Event(enable_timing=True))
-                events["mid"][-1].record(stream)
-                events["axes"].append((a_axis, b_axis, a.numel(), b.numel()))
-            st = L.halo_hadamard_quantize(h._ptr(b), b.shape[0], b.shape[1], b.stride(0), b_axis, BLK, self.qtype,
-                                          h._ptr(qb), qb.stride(0), h._ptr(self.sb), sp)
-            h._check(st, "rotq B")
-            if events is not None:
-                events["gemm"].append(torch.cuda.Event(enable_timing=True))
-                events["gemm"][-1].record(stream)
-            a_major = h.HALO_MAJOR_K if a_axis == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
-            b_major = h.HALO_MAJOR_K if b_axis == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
-            otype = h.HALO_OUT_FP32 if c.dtype == torch.float32 else h.HALO_OUT_BF16
-            st = L.halo_qgemm(h._ptr(qa), h._ptr(self.sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(self.sb),
-                              b_major, qb.stride(0), m, n, k, self.qtype, h._ptr(c), otype, c.stride(0), sp)
-            h._check(st, "qgemm")
-            if events is not None:
-                events["end"].append(torch.cuda.Event(enable_timing=True))
-                events["end"][-1].record(stream)
-            launches += 3
-        return launches
+                ev = torch.cuda.Event(enable_timing=True)
+                ev.record(stream)
+                events.append(ev)
+            if op[0] == "rotq":
+                _, x, ax, q, sc = op
+                st = L.halo_hadamard_quantize(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), ax, BLK, self.qtype,
+                                              h._ptr(q), q.stride(0), h._ptr(sc), sp)
+                h._check(st, "halo_hadamard_quantize")
+            else:
+                _, (qa, sa, ax_a), (qb, sb, ax_b), m, n, k, c = op
+                a_major = h.HALO_MAJOR_K if ax_a == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
+                b_major = h.HALO_MAJOR_K if ax_b == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
+                otype = h.HALO_OUT_FP32 if c.dtype == torch.float32 else h.HALO_OUT_BF16
+                st = L.halo_qgemm(h._ptr(qa), h._ptr(sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(sb), b_major,
+                                  qb.stride(0), m, n, k, self.qtype, h._ptr(c), otype, c.stride(0), sp)
+                h._check(st, "halo_qgemm")
+        if events is not None:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record(stream)
+            events.append(ev)
+        return len(plan)
+
+    def attribute(self, events, steps):
+        """Per-launch durations from an instrumented run of `steps` steps:
+        (gemm ms, [rotq ms, elements] per axis)."""
+        plan = self.plan()
+        gemm_ms, by_axis = 0.0, {0: [0.0, 0], 1: [0.0, 0]}
+        per = len(plan) + 1
+        for s_i in range(steps):
+            evs = events[s_i * per:(s_i + 1) * per]
+            for j, op in enumerate(plan):
+                dt = evs[j].elapsed_time(evs[j + 1])
+                if op[0] == "gemm":
+                    gemm_ms += dt
+                else:
+                    by_axis[op[2]][0] += dt
+                    by_axis[op[2]][1] += op[1].numel()
+        return gemm_ms, by_axis
 
     def rotq_bytes(self) -> int:
-        """Algorithmic bytes of all rotate+quantise launches of one step:
-        bf16 in (2 B) + code out (1 B) per element + one fp32 scale per group."""
+        """Algorithmic bytes of the step's rotate+quantise launches: bf16 in
+        (2 B) + code out (1 B) per element + one fp32 scale per group."""
         h = self.halo
         total = 0
-        for kind, name, a, a_axis, b, b_axis, m, n, k, c in self.gemms():
-            for x, axis in ((a, a_axis), (b, b_axis)):
-                r, cc = x.shape
-                groups = r if axis == h.HALO_AXIS_COLS else cc
-                total += 3 * r * cc + 4 * groups
+        for op in self.plan():
+            if op[0] == "rotq":
+                x, ax = op[1], op[2]
+                groups = x.shape[0] if ax == h.HALO_AXIS_COLS else x.shape[1]
+                total += 3 * x.numel() + 4 * groups
         return total
 
     def gemm_ops(self) -> int:
-        return sum(2 * m * n * k for _, _, _, _, _, _, m, n, k, _ in self.gemms())
+        return sum(2 * op[3] * op[4] * op[5] for op in self.plan() if op[0] == "gemm")
 
 
 def e2e_run(step: LayerStep, steps: int):
@@ -383,7 +435,7 @@ def main():
     if st != halo.HALO_OK:
         raise RuntimeError(f"device error after warm-up at site {site:#x}")
 
-    events = {"rotq": [], "mid": [], "gemm": [], "end": [], "axes": []}
+    # Timed region: K plain steps (no events between launches).
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -393,7 +445,7 @@ def main():
         start.record(stream)
         launches = 0
         for _ in range(args.steps):
-            launches += step.run(events)
+            launches += step.run()
         end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -407,16 +459,17 @@ def main():
     if st != halo.HALO_OK:
         raise RuntimeError(f"device error in the timed region at site {site:#x}")
 
-    rotq_ms = sum(a.elapsed_time(b) for a, b in zip(events["rotq"], events["gemm"]))
-    # per rotation direction: [ms, elements] for axis COLS (rotq_rows kernel) and ROWS (rotq_cols kernels)
-    by_axis = {0: [0.0, 0], 1: [0.0, 0]}
-    for e0, e1, e2, (ax_a, ax_b, na, nb) in zip(events["rotq"], events["mid"], events["gemm"], events["axes"]):
-        by_axis[ax_a][0] += e0.elapsed_time(e1)
-        by_axis[ax_a][1] += na
-        by_axis[ax_b][0] += e1.elapsed_time(e2)
-        by_axis[ax_b][1] += nb
-    gemm_ms = sum(a.elapsed_time(b) for a, b in zip(events["gemm"], events["end"]))
-    n_gemm = len(events["gemm"])
+    # Attribution: the same K steps again with a CUDA event before every launch
+    # (same stream), for the per-kernel durations.
+    events = []
+    for _ in range(args.steps):
+        step.run(events)
+    torch.cuda.synchronize()
+    gemm_ms, by_axis = step.attribute(events, args.steps)
+    ms_instrumented = events[0].elapsed_time(events[-1]) / args.steps
+    rotq_ms = by_axis[0][0] + by_axis[1][0]
+    n_gemm = sum(1 for op in step.plan() if op[0] == "gemm") * args.steps
+
     ops_step = step.ops_per_step()
     ms_step = ms_total / args.steps
     value = ops_step * args.steps * world / (ms_total * 1e-3) / 1e12
@@ -427,21 +480,25 @@ def main():
     # 8-bit : bf16 ratio (4.5 : 2.25); sustained figure, the GEMMs run inside a long step.
     peak8 = 2.0 * pk["bf16_sustained"]
 
+    def gbs(axis):
+        return 3 * by_axis[axis][1] / max(by_axis[axis][0] * 1e-3, 1e-12) / 1e9
+
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8" if qtype == halo.HALO_Q_INT8 else "e4m3",
             "data": "synthetic", "config": config,
             "gpu_launches": launches,
-            "roofline": {"bound": "tensor", "kernel": "qgemm_kernel", "achieved": gemm_tops, "peak": peak8,
+            "roofline": {"bound": "tensor", "kernel": "qgemm_pair_kernel", "achieved": gemm_tops, "peak": peak8,
                          "unit": "TFLOP/s", "frac": gemm_tops / peak8, "traffic": None,
-                         "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']})",
+                         "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']}); "
+                                      f"burst 2 x {pk['bf16']} = {2 * pk['bf16']:.1f}",
                          "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
             "rotq": {"gbs": rotq_gbs, "peak_gbs": pk["hbm_gbs"], "frac": rotq_gbs / pk["hbm_gbs"],
                      "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps,
-                     "along_contiguous_dim_gbs": 3 * by_axis[0][1] / max(by_axis[0][0] * 1e-3, 1e-12) / 1e9,
-                     "along_dim0_gbs": 3 * by_axis[1][1] / max(by_axis[1][0] * 1e-3, 1e-12) / 1e9,
+                     "along_contiguous_dim_gbs": gbs(0), "along_dim0_gbs": gbs(1),
                      "along_contiguous_dim_ms_per_step": by_axis[0][0] / args.steps,
                      "along_dim0_ms_per_step": by_axis[1][0] / args.steps},
+            "ms_per_step_instrumented": ms_instrumented,
             "clocks": clocks.summary()}
 
     if rank == 0 and not args.no_e2e:

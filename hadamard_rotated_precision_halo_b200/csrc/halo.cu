@@ -145,6 +145,34 @@ halo_status_t noalloc_setup(int dev) {
   return HALO_OK;
 }
 
+// Launch configuration with programmatic dependent launch on (each kernel's
+// prologue may overlap the previous kernel's tail; the kernels wait with
+// griddepcontrol.wait before touching global memory) and an optional cluster
+// shape.  Use in place: cfg points into this object.
+struct Launch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster_x) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = cluster_x;
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+  }
+};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
@@ -168,18 +196,17 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
 halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
                                void* q, int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
   const int nb = static_cast<int>(cols / 128);
-  // About 128 chunks per tile; a tile always holds whole rows (for blk 256, nb
-  // is even, so the two chunks of a block sit on adjacent lanes).
-  const int nr = std::max(1, 128 / nb);
-  const int active = nr * nb;
-  const int threads = (active + 31) / 32 * 32;
-  const int num_tiles = static_cast<int>((rows + nr - 1) / nr);
+  // A row group of ceil(nb / 32) warps owns one row at a time; 4 warps per
+  // CTA when a group fits in 4, else one group per CTA (up to 8 warps).
+  const int gw = (nb + 31) / 32;
+  const int groups = gw <= 4 ? 4 / gw : 1;
+  const int threads = groups * gw * 32;
 
   CUtensorMap tm_x, tm_q;
   {
     cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
-    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(nb), static_cast<cuuint32_t>(nr)};
+    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(nb), 1};
     halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != HALO_OK) return st;
@@ -187,21 +214,19 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   {
     cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(ld_q)};
-    cuuint32_t box[3] = {kRowsOutSlot, static_cast<cuuint32_t>(nb), static_cast<cuuint32_t>(nr)};
+    cuuint32_t box[3] = {kRowsOutSlot, static_cast<cuuint32_t>(nb), 1};
     halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != HALO_OK) return st;
   }
-  const size_t in_stride = (static_cast<size_t>(active) * kRowsInSlot + 127) & ~size_t(127);
-  const size_t out_stride = (static_cast<size_t>(active) * kRowsOutSlot + 127) & ~size_t(127);
-  const size_t smem = 2 * in_stride + 2 * out_stride + 128;  // + alignment slack
+  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw) + 128;  // + alignment slack
 
   RotqRowsParams p;
   p.scales = scales;
   p.rows = rows;
   p.nb = nb;
-  p.nr = nr;
-  p.num_tiles = num_tiles;
+  p.gw = gw;
+  p.groups = groups;
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(static_cast<double>(blk))));
 
@@ -213,9 +238,10 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   int per_sm = 0;
   HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
   if (per_sm < 1) per_sm = 1;
-  const int grid = static_cast<int>(std::min<int64_t>(num_tiles, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
-  kern<<<grid, threads, smem, stream>>>(tm_x, tm_q, p);
-  HALO_CUDA(cudaGetLastError());
+  const int64_t ctas_needed = (rows + groups - 1) / groups;
+  const int grid = static_cast<int>(std::min<int64_t>(ctas_needed, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
+  Launch L(dim3(grid), dim3(threads), smem, stream, 0);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
   return HALO_OK;
 }
 
@@ -249,32 +275,23 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
   Cols1Kernel kern = cols_1pass_kernel(qtype, nw);
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(32 * nw, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(nw) * (2 * kColsInBytes + kColsOutBytes) + 128;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   // Persistent: as many clusters as fit at once (each loops over strips).
-  cfg.gridDim = dim3(cl, 1, 1);
+  Launch L(dim3(cl, 1, 1), dim3(32 * nw), static_cast<size_t>(nw) * (2 * kColsInBytes + kColsOutBytes) + 128,
+           stream, cl);
   int max_clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1) {
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &L.cfg) != cudaSuccess || max_clusters < 1) {
     (void)cudaGetLastError();
     max_clusters = std::max(1, g_dev[dev].sm_count / cl);
   }
-  cfg.gridDim = dim3(cl, std::min(strips, max_clusters), 1);
-  HALO_CUDA(cudaLaunchKernelEx(&cfg, kern, tm_x, tm_q, p));
+  L.cfg.gridDim = dim3(cl, std::min(strips, max_clusters), 1);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
   return HALO_OK;
 }
 
 halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
                                int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
   const int nblocks = static_cast<int>(rows / 128);
+  // Most warps per CTA (up to 4) with at most 16 CTAs per cluster.
   for (int nw = 4; nw >= 1; --nw) {
     if (nblocks % nw == 0 && nblocks / nw <= 16)
       return launch_rotq_cols_1pass(x, rows, cols, ld_x, qtype, q, ld_q, scales, stream, nw, nblocks / nw, dev);
@@ -311,22 +328,11 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
   const size_t smem = static_cast<size_t>(warps) * (kColsStages * kColsInBytes + 2 * kColsOutBytes) + 128;
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cl, strips, 1);
-  cfg.blockDim = dim3(32 * warps, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  Launch L(dim3(cl, strips, 1), dim3(32 * warps), smem, stream, cl);
   if (qtype == HALO_Q_INT8)
-    HALO_CUDA(cudaLaunchKernelEx(&cfg, rotq_cols_kernel<0>, tm_x, tm_q, p));
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, rotq_cols_kernel<0>, tm_x, tm_q, p));
   else
-    HALO_CUDA(cudaLaunchKernelEx(&cfg, rotq_cols_kernel<1>, tm_x, tm_q, p));
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, rotq_cols_kernel<1>, tm_x, tm_q, p));
   return HALO_OK;
 }
 
@@ -399,30 +405,19 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
   p.out_bf16 = otype == HALO_OUT_BF16;
   if (!use_pair) {
     const int grid = std::min(p.num_tiles, g_dev[dev].sm_count);
+    Launch L(dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, stream, 0);
     if (qtype == HALO_Q_INT8)
-      qgemm_kernel<0><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
+      HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_kernel<0>, tm_a, tm_b, p));
     else
-      qgemm_kernel<1><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tm_a, tm_b, p);
-    HALO_CUDA(cudaGetLastError());
+      HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_kernel<1>, tm_a, tm_b, p));
     return HALO_OK;
   }
   const int pairs = std::min(p.num_tiles, g_dev[dev].sm_count / 2);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPairSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  Launch L(dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, stream, 2);
   if (qtype == HALO_Q_INT8)
-    HALO_CUDA(cudaLaunchKernelEx(&cfg, qgemm_pair_kernel<0>, tm_a, tm_b, p));
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_pair_kernel<0>, tm_a, tm_b, p));
   else
-    HALO_CUDA(cudaLaunchKernelEx(&cfg, qgemm_pair_kernel<1>, tm_a, tm_b, p));
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_pair_kernel<1>, tm_a, tm_b, p));
   return HALO_OK;
 }
 

@@ -79,6 +79,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigne
   }
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Wait until the preceding kernel in the stream has completed and its memory is
+// visible (returns at once when the launch has no programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel in the stream begin launching (its prologue overlaps our
+// tail; it still waits in griddep_wait() for our completion before touching
+// memory).  Used only by kernels whose whole grid is resident from the start.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- barriers
 // Block-wide OR vote on a named barrier (all `nthreads` threads of the named
 // barrier must take part).

@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int kblocks = (p.k + kGemmBK - 1) / kGemmBK;
+  griddep_wait();  // codes and scales written, output read, by the previous kernels
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -324,6 +326,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int kblocks = (p.k + kGemmBK - 1) / kGemmBK;
+  griddep_wait();  // codes and scales written, output read, by the previous kernels
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {

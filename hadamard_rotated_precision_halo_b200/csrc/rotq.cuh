@@ -42,16 +42,6 @@ enum : unsigned int {
 constexpr int kRowsInSlot = 272;   // bytes (136 bf16)
 constexpr int kRowsOutSlot = 144;  // bytes
 
-struct RotqRowsParams {
-  float* scales;
-  int64_t rows;
-  int nb;          // 128-element chunks per row (cols / 128)
-  int nr;          // rows per tile
-  int num_tiles;   // ceil(rows / nr)
-  float qmax;
-  float scale_mult;  // 1 / (qmax * sqrt(blk))
-};
-
 __device__ __forceinline__ float2 f2_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.f, -1.f), a);
@@ -84,6 +74,40 @@ __device__ __forceinline__ void fwht128_pairs(float2 (&v)[64]) {
   }
 }
 
+// max |v| over 128 values as a balanced tree (depth 7 instead of a 128-long
+// dependency chain; fmaxf chains are not reassociated by the compiler).
+__device__ __forceinline__ float absmax128(const float2 (&v)[64]) {
+  float m[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    m[i] = fmaxf(fmaxf(fabsf(v[2 * i].x), fabsf(v[2 * i].y)), fmaxf(fabsf(v[2 * i + 1].x), fabsf(v[2 * i + 1].y)));
+#pragma unroll
+  for (int w = 16; w >= 1; w /= 2) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  }
+  return m[0];
+}
+
+// Column-wise max |v| of 64 float2 (x and y are two columns), as trees.
+__device__ __forceinline__ float2 absmax64_cols(const float2 (&v)[64]) {
+  float mx[32], my[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    mx[i] = fmaxf(fabsf(v[2 * i].x), fabsf(v[2 * i + 1].x));
+    my[i] = fmaxf(fabsf(v[2 * i].y), fabsf(v[2 * i + 1].y));
+  }
+#pragma unroll
+  for (int w = 16; w >= 1; w /= 2) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      mx[i] = fmaxf(mx[i], mx[i + w]);
+      my[i] = fmaxf(my[i], my[i + w]);
+    }
+  }
+  return make_float2(mx[0], my[0]);
+}
+
 // Round-half-even of t (|t| <= 2^22) to an int8 code in the low byte of the
 // returned word: adding 1.5 * 2^23 puts the rounded integer into the low
 // mantissa bits (round-to-nearest-even of the fused multiply-add).
@@ -102,100 +126,121 @@ __device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
 }
 
 // ------------------------------------------------------------------------------------------
-// rotq_rows: one thread owns one 128-element chunk of one row.  A tile is `nr`
-// whole rows (nr * nb chunks <= blockDim.x).  The tile arrives by one 3-D TMA
-// load of the view [rows][nb][128] with a 136-element box along the innermost
-// dimension: the 8 elements past each chunk fall outside the tensor, read as
-// zeros and give the padded slot layout for free.  Codes leave the same way
-// (144-byte box, the out-of-range tail is not written).
+// rotq_rows: one thread owns one 128-element chunk of one row.  A row is
+// handled by a "row group" of G = ceil(nb / 32) warps (one warp when the row
+// has 4096 elements); a CTA holds 4 / G groups (or one group of G > 4 warps),
+// and every group streams its own rows independently with its own 2-stage TMA
+// ring, so warps do not wait on each other beyond their own row.  A row
+// arrives by one 3-D TMA load of the view [rows][nb][128] with a 136-element
+// box along the innermost dimension: the 8 elements past each chunk fall
+// outside the tensor, read as zeros and give the padded per-thread slot for
+// free.  Codes leave the same way (144-byte box; the out-of-range tail is not
+// written).  Row absmax: redux.sync within a warp, shared memory across the
+// group's warps.
 // ------------------------------------------------------------------------------------------
+struct RotqRowsParams {
+  float* scales;
+  int64_t rows;
+  int nb;        // 128-element chunks per row (cols / 128)
+  int gw;        // warps per row group
+  int groups;    // row groups per CTA
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(blk))
+};
+
+// Shared-memory bytes of one row group: 2 input stages and one code tile.
+__host__ __device__ inline uint32_t rows_group_in_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsInSlot; }
+__host__ __device__ inline uint32_t rows_group_out_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsOutSlot; }
+__host__ __device__ inline uint32_t rows_group_smem(int gw) { return 2 * rows_group_in_bytes(gw) + rows_group_out_bytes(gw); }
+
+__device__ __forceinline__ void group_sync(int gw, int grp) {
+  if (gw == 1)
+    __syncwarp();
+  else
+    named_bar_sync(1 + grp, gw * 32);
+}
+
 template <int BLK, int QT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256)
     rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                      RotqRowsParams p) {
-  constexpr int kStages = 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ uint64_t full_bar[kStages];
-  __shared__ uint32_t s_amax[2][256];
+  __shared__ uint64_t full_bar[8][2];
+  __shared__ uint32_t s_wmax[2][8];  // per-warp row maxima, by row parity
 
-  const int tid = threadIdx.x;
-  const int active = p.nr * p.nb;
-  const uint32_t in_bytes = static_cast<uint32_t>(active) * kRowsInSlot;
-  const uint32_t in_stride = (in_bytes + 127u) & ~127u;
-  const uint32_t out_bytes = static_cast<uint32_t>(active) * kRowsOutSlot;
-  const uint32_t out_stride = (out_bytes + 127u) & ~127u;
-  uint8_t* s_in = smem;
-  uint8_t* s_out = smem + kStages * in_stride;
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int gw = p.gw;
+  const int grp = warp / gw;
+  const int wig = warp - grp * gw;          // warp index inside the group
+  const int chunk = wig * 32 + lane;        // this thread's 128-element chunk of the row
+  const bool is_active = chunk < p.nb;
+  const bool leader = (wig == 0 && lane == 0);
+  const uint32_t in_bytes = static_cast<uint32_t>(p.nb) * kRowsInSlot;  // one row's box
+  uint8_t* g_in = smem + grp * rows_group_smem(gw);
+  uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw);
 
-  const int my_row = tid / p.nb;
-  const int my_chunk = tid - my_row * p.nb;
-  const bool is_active = tid < active;
-
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full_bar[s], 1);
+  if (leader) {
+    mbar_init(&full_bar[grp][0], 1);
+    mbar_init(&full_bar[grp][1], 1);
     fence_mbar_init();
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_q);
   }
-  for (int i = tid; i < 2 * 256; i += blockDim.x) (&s_amax[0][0])[i] = 0u;
   __syncthreads();
+  griddep_wait();  // inputs written and codes read by the previous kernel
+  griddep_launch_dependents();
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      const int tile = blockIdx.x + s * gridDim.x;
-      if (tile < p.num_tiles) {
-        mbar_arrive_expect_tx(&full_bar[s], in_bytes);
-        tma_load_3d(s_in + s * in_stride, &tm_x, &full_bar[s], 0, 0, tile * p.nr);
-      }
-    }
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * p.groups + grp;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * p.groups;
+  const int64_t nmine = first < p.rows ? (p.rows - first + step - 1) / step : 0;
+
+  auto issue = [&](int64_t it) {
+    const int st = static_cast<int>(it & 1);
+    mbar_arrive_expect_tx(&full_bar[grp][st], in_bytes);
+    tma_load_3d(g_in + st * rows_group_in_bytes(gw), &tm_x, &full_bar[grp][st], 0, 0,
+                static_cast<int32_t>(first + it * step));
+  };
+  if (leader) {
+    if (nmine > 0) issue(0);
+    if (nmine > 1) issue(1);
   }
 
-  uint32_t it = 0;
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
-    const int s = it % kStages;
-    const uint32_t ph = (it / kStages) & 1u;
-    const int par = it & 1;
-    const bool ok = mbar_wait(&full_bar[s], ph, kSiteRotqRowsLoad);
-    if (__syncthreads_or(!ok)) break;
-
-    uint4 raw[16];
-    if (is_active) {
-      const uint4* src = reinterpret_cast<const uint4*>(s_in + s * in_stride + tid * kRowsInSlot);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) raw[k] = src[k];
+  bool dead = false;  // a load wait ran out: stop waiting and loading, keep every barrier
+  for (int64_t it = 0; it < nmine; ++it) {
+    const int st = static_cast<int>(it & 1);
+    const int par = static_cast<int>(it & 1);
+    const int64_t row = first + it * step;
+    if (!dead) {
+      const bool ok = mbar_wait(&full_bar[grp][st], static_cast<uint32_t>((it >> 1) & 1), kSiteRotqRowsLoad);
+      dead = !ok;
     }
-    __syncthreads();  // stage s fully consumed; code buffer `par` free once the wait below returns
-    if (tid == 0) {
-      const int next = tile + kStages * gridDim.x;
-      if (next < p.num_tiles) {
-        mbar_arrive_expect_tx(&full_bar[s], in_bytes);
-        tma_load_3d(s_in + s * in_stride, &tm_x, &full_bar[s], 0, 0, next * p.nr);
-      }
-      bulk_wait_read<1>();
-    }
-    for (int i = tid; i < p.nr; i += blockDim.x) s_amax[par ^ 1][i] = 0u;
-
     float2 v[64];
-    float amax = 0.f;
-    if (is_active) {
+    if (is_active && !dead) {
+      const uint4* src = reinterpret_cast<const uint4*>(g_in + st * rows_group_in_bytes(gw) + chunk * kRowsInSlot);
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        v[4 * k + 0] = bf16x2_to_f2(raw[k].x);
-        v[4 * k + 1] = bf16x2_to_f2(raw[k].y);
-        v[4 * k + 2] = bf16x2_to_f2(raw[k].z);
-        v[4 * k + 3] = bf16x2_to_f2(raw[k].w);
+        const uint4 raw = src[k];
+        v[4 * k + 0] = bf16x2_to_f2(raw.x);
+        v[4 * k + 1] = bf16x2_to_f2(raw.y);
+        v[4 * k + 2] = bf16x2_to_f2(raw.z);
+        v[4 * k + 3] = bf16x2_to_f2(raw.w);
       }
       fwht128_pairs(v);
     } else {
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
     }
+    group_sync(gw, grp);  // stage `st` fully read
+    if (leader) {
+      if (!dead && it + 2 < nmine) issue(it + 2);
+      bulk_wait_read<0>();  // the previous row's store has read the code tile
+    }
     if (BLK == 256) {
-      // Top stage of the 256-point transform: chunk pairs (2j, 2j+1) of a row
-      // sit on adjacent lanes.  Lower half keeps a + b, upper half a - b.
-      // Every lane of the warp takes part (idle lanes carry zeros).
-      const bool upper = (my_chunk & 1) != 0;
+      // Top stage of the 256-point transform: chunk pairs (2j, 2j+1) sit on
+      // adjacent lanes.  Lower half keeps a + b, upper half a - b.
+      const bool upper = (chunk & 1) != 0;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         float2 o;
@@ -204,19 +249,20 @@ __global__ void __launch_bounds__(256, 1)
         v[i] = upper ? f2_sub(o, v[i]) : f2_add(v[i], o);
       }
     }
-    if (is_active) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
-      atomicMax(&s_amax[par][my_row], __float_as_uint(amax));
+    const float amax = absmax128(v);
+    uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if (gw > 1) {
+      if (lane == 0) s_wmax[par][warp] = wmax;
+      group_sync(gw, grp);  // also orders the leader's store wait before the code writes
+      for (int w = 0; w < gw; ++w) wmax = max(wmax, s_wmax[par][grp * gw + w]);
+    } else {
+      __syncwarp();
     }
-    __syncthreads();
-
+    const float row_amax = __uint_as_float(wmax);
+    const float r = row_amax > 0.f ? __fdiv_rn(p.qmax, row_amax) : 0.f;
+    if (chunk == 0) p.scales[row] = row_amax * p.scale_mult;
     if (is_active) {
-      const float row_amax = __uint_as_float(s_amax[par][my_row]);
-      const float r = row_amax > 0.f ? __fdiv_rn(p.qmax, row_amax) : 0.f;
-      const int64_t grow = static_cast<int64_t>(tile) * p.nr + my_row;
-      if (my_chunk == 0 && grow < p.rows) p.scales[grow] = row_amax * p.scale_mult;
-      uint4* dst = reinterpret_cast<uint4*>(s_out + par * out_stride + tid * kRowsOutSlot);
+      uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         uint32_t w[4];
@@ -235,26 +281,15 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tma_store_3d(&tm_q, s_out + par * out_stride, 0, 0, tile * p.nr);
+    group_sync(gw, grp);
+    if (leader) {
+      tma_store_3d(&tm_q, g_out, 0, 0, static_cast<int32_t>(row));
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait<0>();
+  if (leader) bulk_wait<0>();
 }
 
-// ------------------------------------------------------------------------------------------
-// rotq_cols: rotation along dimension 0.  A cluster of CTAs covers one strip
-// of 32 columns over all rows; its CTAs split the 128-row blocks of the strip.
-// Lane (p, h) of a warp owns columns (2p, 2p+1) of the strip and the 64 rows
-// of a 128-row block with row parity h; the bottom butterfly stage is formed
-// while loading (each lane reads both rows of a pair), the other six run on
-// the lane's own rows.  The column maximum needs the whole column, so the
-// strip is streamed twice: pass 1 reduces the maxima (warp -> CTA -> cluster
-// through distributed shared memory), pass 2 re-reads the strip (an L2 hit:
-// a cluster's strip is at most a few MB) and writes the codes.
-// ------------------------------------------------------------------------------------------
 constexpr int kColsStrip = 32;
 constexpr int kColsInBytes = 128 * kColsStrip * 2;  // one 128 x 32 bf16 block
 constexpr int kColsOutBytes = 128 * kColsStrip;     // one 128 x 32 block of codes
@@ -342,6 +377,7 @@ __global__ void __launch_bounds__(128)
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();  // not resident all at once: no early launch of dependents
 
   // This warp's blocks: b_i = crank + csize * (warp + warps * i).
   const int first = static_cast<int>(crank) + static_cast<int>(csize) * warp;
@@ -384,11 +420,9 @@ __global__ void __launch_bounds__(128)
     __syncwarp();
     if (lane == 0 && j + kColsStages < nseq) issue(j + kColsStages);
     cols_fwht_rest(v);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      m0 = fmaxf(m0, fabsf(v[i].x));
-      m1 = fmaxf(m1, fabsf(v[i].y));
-    }
+    const float2 mm = absmax64_cols(v);
+    m0 = fmaxf(m0, mm.x);
+    m1 = fmaxf(m1, mm.y);
   }
   // Cluster-wide column maxima through distributed shared memory.
   __syncthreads();
@@ -511,6 +545,8 @@ __global__ void __launch_bounds__(NW * 32)
   }
   cluster_arrive();  // every peer is running and initialised before the first remote store
   cluster_wait();
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int first = blockIdx.y;
   const int step = gridDim.y;
@@ -544,12 +580,8 @@ __global__ void __launch_bounds__(NW * 32)
     __syncwarp();
     if (lane == 0 && !dead && k + 2 < nmine) issue(k + 2);
     cols_fwht_rest(v);
-    float m0 = 0.f, m1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      m0 = fmaxf(m0, fabsf(v[i].x));
-      m1 = fmaxf(m1, fabsf(v[i].y));
-    }
+    const float2 mm = absmax64_cols(v);
+    float m0 = mm.x, m1 = mm.y;
     m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
     m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
     if (h == 0) {
