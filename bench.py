@@ -364,11 +364,122 @@ def cpu_baseline(seconds_target: float = 15.0):
             "sample": s.describe(dt)}
 
 
+# ---------------------------------------------------------- auxiliary measurements
+def _clock_proc():
+    return subprocess.Popen(["nvidia-smi", "-i", str(torch.cuda.current_device()),
+                             "--query-gpu=clocks.sm,power.draw", "--format=csv,noheader,nounits", "-lms", "50"],
+                            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+
+def _clock_stop(p):
+    p.terminate()
+    out, _ = p.communicate()
+    vals = [l.split(",") for l in out.splitlines() if l.strip()]
+    sm = sorted(float(v[0]) for v in vals)
+    pw = sorted(float(v[1]) for v in vals)
+    return (sm[len(sm) // 2] if sm else None), (pw[len(pw) // 2] if pw else None)
+
+
+def measure_peaks(n: int = 8192, seconds: float = 3.0):
+    """8-bit GEMM throughput at n^3 on this GPU: this library's halo_qgemm next to
+    cuBLAS (torch._int_mm for INT8, torch._scaled_mm for FP8), best of 10 single
+    launches (burst) and a `seconds`-long back-to-back loop (sustained, with the
+    SM clock and power seen meanwhile).  Library GEMMs are the comparison here,
+    not part of the product path."""
+    import hadamard_rotated_precision_halo_b200 as halo
+
+    g = torch.Generator(device="cuda").manual_seed(0)
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda", generator=g)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda", generator=g)
+    a8 = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+    b8 = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+    ones = torch.ones(n, dtype=torch.float32, device="cuda")
+    one = torch.ones((), device="cuda")
+    c = torch.empty((n, n), dtype=torch.bfloat16, device="cuda")
+    cases = {
+        "halo_int8": lambda: halo.halo_qgemm(a, ones, 0, b, ones, 0, n, n, n, 0, 1, c=c),
+        "cublas_int8": lambda: torch._int_mm(a, b.t()),
+        "halo_e4m3": lambda: halo.halo_qgemm(a8, ones, 0, b8, ones, 0, n, n, n, 1, 1, c=c),
+        "cublas_e4m3": lambda: torch._scaled_mm(a8, b8.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+    }
+    out = {}
+    for name, fn in cases.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        best = 1e30
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        proc = _clock_proc()
+        time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        t0, cnt = time.time(), 0
+        while time.time() - t0 < seconds:
+            for _ in range(20):
+                fn()
+            cnt += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        sm, pw = _clock_stop(proc)
+        out[name] = {"burst_tops": 2 * n ** 3 / (best * 1e-3) / 1e12,
+                     "sustained_tops": 2 * n ** 3 * cnt / (e0.elapsed_time(e1) * 1e-3) / 1e12,
+                     "sm_mhz_median": sm, "power_w_median": pw}
+    return {"measure": "8-bit GEMM peaks", "n": n, "results": out}
+
+
+ROTQ_SHAPES = {  # (rows, cols) of every rotate+quantise operand of the 70B layer, and the standalone case
+    "along_contiguous_dim": [(4096, 8192), (8192, 8192), (1024, 8192), (28672, 8192), (4096, 28672),
+                             (8192, 28672), (4096, 1024), (16384, 4096)],
+    "along_dim0": [(8192, 8192), (1024, 8192), (28672, 8192), (8192, 28672), (4096, 8192), (4096, 28672),
+                   (4096, 1024), (16384, 4096)],
+}
+
+
+def measure_rotq_shapes(repeats: int = 10):
+    """halo_hadamard_quantize on each shape alone (INT8 and E4M3, block 128), a
+    512 MB write between repeats to flush L2; median time and algorithmic GB/s
+    (3 B per element + 4 B per scale)."""
+    import hadamard_rotated_precision_halo_b200 as halo
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    out = []
+    for name, shapes in ROTQ_SHAPES.items():
+        axis = halo.HALO_AXIS_COLS if name == "along_contiguous_dim" else halo.HALO_AXIS_ROWS
+        for r, c in shapes:
+            x = inputs.activations(r, c, seed=1, device="cuda")
+            for qt in (halo.HALO_Q_INT8, halo.HALO_Q_E4M3):
+                q, sc = halo.halo_hadamard_quantize(x, axis, BLK, qt)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(repeats):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    halo.halo_hadamard_quantize(x, axis, BLK, qt, q_out=q, scales_out=sc)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                ms = sorted(ts)[len(ts) // 2]
+                nbytes = 3 * x.numel() + 4 * sc.numel()
+                out.append({"direction": name, "shape": [r, c], "qtype": "int8" if qt == 0 else "e4m3",
+                            "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
+            del x, q, sc
+    return {"measure": "rotate+quantise per shape", "block": BLK, "results": out}
+
+
 # ------------------------------------------------------------------------- main
 WORKLOADS = {
     "llama70b_layer_fwd_bwd": (inputs.LLAMA70B_LAYER, ("fwd", "dx", "dw")),
     "llama7b_attn_proj_fwd": (inputs.LLAMA7B_ATTN_PROJ, ("fwd",)),
     "llama7b_ffn_down_bwd": (inputs.LLAMA7B_FFN_DOWN, ("dx", "dw")),
+    "llama70b_gate_proj_dx": (inputs.LLAMA70B_GATE, ("dx",)),
 }
 
 
@@ -383,7 +494,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama70b_layer_fwd_bwd", choices=sorted(WORKLOADS),
                     help="the bench line uses the default; the single-GEMM cases serve profiling")
+    ap.add_argument("--measure-peaks", action="store_true",
+                    help="print 8-bit GEMM burst / sustained throughput (this library and cuBLAS) and exit")
+    ap.add_argument("--rotq-shapes", action="store_true",
+                    help="print rotate+quantise time per operand shape of the layer and exit")
     args = ap.parse_args()
+    if args.measure_peaks or args.rotq_shapes:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(measure_peaks() if args.measure_peaks else measure_rotq_shapes()), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -13,7 +13,7 @@ import torch
 import hadamard_rotated_precision_halo_b200 as halo
 import oracle
 from hadamard_rotated_precision_halo_b200 import inputs
-from tests._parity import OUT_REL, check_codes, check_output, oracle_operand, u8
+from tests._parity import check_codes, check_output, oracle_operand
 
 pytestmark = pytest.mark.gpu
 
@@ -250,3 +250,28 @@ def test_full_backward_8192x11008x4096():
     ni_t, ki_t = torch.from_numpy(ni).cuda(), torch.from_numpy(ki).cuda()
     ref = _sampled_gemm_ref(dy[:, ni_t].cpu(), 0, x[:, ki_t].cpu(), 0, 128, INT8)
     check_output(dw[ni_t][:, ki_t], ref)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+def test_full_llama70b_layer_step_as_benchmarked(qtype):
+    """The Llama-70B layer step (4096 tokens; q, k, v, o, gate, up, down; forward,
+    dX and dW) run exactly as bench.py times it -- the same launches, with the
+    attention and MLP inputs rotated once and shared -- and every one of the 21
+    outputs checked on sampled rows x columns against the oracle."""
+    import bench
+
+    step = bench.LayerStep(inputs.LLAMA70B_LAYER, seed=4, device=torch.device("cuda"), qtype=qtype)
+    step.run()
+    torch.cuda.synchronize()
+    for gi, (kind, name, a, a_axis, b, b_axis, m, n, k, c) in enumerate(step.gemms()):
+        ri, cj = _sample(m, 8, 100 + gi), _sample(n, 16, 200 + gi)
+        ri_t, cj_t = torch.from_numpy(ri).cuda(), torch.from_numpy(cj).cuda()
+        # logical rows of A (B) are rows of its storage when rotated along the
+        # contiguous dim, columns of its storage when rotated along dim 0
+        a_s = a[ri_t] if a_axis == COLS else a[:, ri_t]
+        b_s = b[cj_t] if b_axis == COLS else b[:, cj_t]
+        ref = _sampled_gemm_ref(a_s.cpu(), 1 if a_axis == COLS else 0, b_s.cpu(), 1 if b_axis == COLS else 0, 128,
+                                qtype)
+        check_output(c[ri_t][:, cj_t], ref)
+    del step
+    torch.cuda.empty_cache()
