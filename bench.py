@@ -35,6 +35,11 @@ if ROOT not in sys.path:
 from hadamard_rotated_precision_halo_b200 import inputs  # noqa: E402
 
 METRIC = "rotated-qGEMM TOPS & rotate+quant GB/s at Llama shapes vs B200 peak (1 GPU)"
+# DRAM bytes (read + write) per qgemm_pair_kernel launch, averaged over the 21
+# GEMMs of the INT8 layer step, from one ncu capture of the current kernel
+# (profiles/qgemm_pair_kernel_llama70b_layer_traffic.md).  Set to None when the
+# kernel changes until it is captured again.
+GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER = 485.9e6
 UNIT = "TOPS"
 BLK = 128
 
@@ -265,6 +270,16 @@ class LayerStep:
                 x, ax = op[1], op[2]
                 groups = x.shape[0] if ax == h.HALO_AXIS_COLS else x.shape[1]
                 total += 3 * x.numel() + 4 * groups
+        return total
+
+    def gemm_bytes(self) -> int:
+        """Algorithmic DRAM bytes of the step's GEMMs: both code operands, the
+        output and the two scale vectors."""
+        total = 0
+        for op in self.plan():
+            if op[0] == "gemm":
+                m, n, k, c = op[3], op[4], op[5], op[6]
+                total += m * k + n * k + m * n * c.element_size() + 4 * (m + n)
         return total
 
     def gemm_ops(self) -> int:
@@ -608,7 +623,11 @@ def main():
             "data": "synthetic", "config": config,
             "gpu_launches": launches,
             "roofline": {"bound": "tensor", "kernel": "qgemm_pair_kernel", "achieved": gemm_tops, "peak": peak8,
-                         "unit": "TFLOP/s", "frac": gemm_tops / peak8, "traffic": None,
+                         "unit": "TFLOP/s", "frac": gemm_tops / peak8,
+                         "traffic": (GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER
+                                     if args.workload == "llama70b_layer_fwd_bwd" and args.qtype == "int8" else None),
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                         "algorithmic_bytes_per_launch": step.gemm_bytes() / max(n_gemm // args.steps, 1),
                          "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']}); "
                                       f"burst 2 x {pk['bf16']} = {2 * pk['bf16']:.1f}",
                          "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
