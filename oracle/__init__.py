@@ -61,6 +61,9 @@ def _load():
         "halo_oracle_e4m3_decode_array": (None, [P, I64, P]),
         "halo_oracle_boundary_distance_array": (None, [P, I64, I, P]),
         "halo_oracle_quantize": (None, [P, I64, I64, I, I, P, P, P]),
+        "halo_oracle_rotate_signed_along_cols": (None, [P, I64, I64, I64, I64, P, P]),
+        "halo_oracle_rotate_signed_along_rows": (None, [P, I64, I64, I64, I64, P, P]),
+        "halo_oracle_quantize_stochastic": (None, [P, I64, I64, I, I, P, P, P, P]),
         "halo_oracle_gemm_i8": (None, [P, P, I64, I64, I64, P]),
         "halo_oracle_gemm_e4m3": (None, [P, P, I64, I64, I64, P]),
         "halo_oracle_dequant": (None, [P, P, P, I64, I64, P]),
@@ -136,6 +139,36 @@ def rotate(x, blk: int, axis: int) -> np.ndarray:
         assert rows % blk == 0
         lib.halo_oracle_rotate_along_rows(_ptr(xb), rows, cols, cols, blk, _ptr(out))
     return out
+
+
+def rotate_signed(x, blk: int, axis: int, signs) -> np.ndarray:
+    """Random-sign rotation H (D x): each element times the +-1 sign of its
+    position along the rotated dimension, then the block transform."""
+    xb = _bf16_bits(x)
+    rows, cols = xb.shape
+    sg = np.ascontiguousarray(signs, dtype=np.int8)
+    assert sg.shape == ((cols,) if axis == 1 else (rows,))
+    out = np.empty((rows, cols), dtype=np.float64)
+    lib = _load()
+    if axis == 1:
+        lib.halo_oracle_rotate_signed_along_cols(_ptr(xb), rows, cols, cols, blk, _ptr(sg), _ptr(out))
+    else:
+        lib.halo_oracle_rotate_signed_along_rows(_ptr(xb), rows, cols, cols, blk, _ptr(sg), _ptr(out))
+    return out
+
+
+def quantize_stochastic(v: np.ndarray, axis: int, qtype: int, rand_bits):
+    """Stochastic-rounding quantiser: u = rand_bits / 65536 per element (uint16, layout of v)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, cols = v.shape
+    rb = np.ascontiguousarray(rand_bits, dtype=np.uint16)
+    assert rb.shape == v.shape
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    scales = np.empty(rows if axis == 0 else cols, dtype=np.float32)
+    t = np.empty((rows, cols), dtype=np.float64)
+    _load().halo_oracle_quantize_stochastic(_ptr(v), rows, cols, axis, qtype, _ptr(rb), _ptr(codes), _ptr(scales),
+                                            _ptr(t))
+    return codes, scales, t
 
 
 def quantize(v: np.ndarray, axis: int, qtype: int):

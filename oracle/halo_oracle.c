@@ -104,6 +104,35 @@ void halo_oracle_rotate_along_rows(const uint16_t* x, int64_t rows, int64_t cols
   free(col);
 }
 
+/* Random-sign variant of the two rotations above: every element is first
+ * multiplied by the sign assigned to its position along the rotated
+ * dimension (signs[c] for the contiguous dimension, signs[r] for dimension 0,
+ * each +1 or -1), then transformed: H (D x) with D = diag(signs).  The same
+ * signs on both GEMM operands keep the product, since (H D)^T (H D) = I
+ * [HALO blog page sec. 4.2: every node seeds the Hadamard matrix alike]. */
+void halo_oracle_rotate_signed_along_cols(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                          int64_t blk, const int8_t* signs, double* v) {
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c)
+      v[r * cols + c] = (double)signs[c] * halo_oracle_bf16_to_f64(x[r * ld + c]);
+    for (int64_t c0 = 0; c0 < cols; c0 += blk) halo_oracle_fwht(&v[r * cols + c0], blk);
+  }
+}
+
+void halo_oracle_rotate_signed_along_rows(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                          int64_t blk, const int8_t* signs, double* v) {
+  double* col = (double*)malloc(sizeof(double) * (size_t)blk);
+  for (int64_t c = 0; c < cols; ++c) {
+    for (int64_t r0 = 0; r0 < rows; r0 += blk) {
+      for (int64_t i = 0; i < blk; ++i)
+        col[i] = (double)signs[r0 + i] * halo_oracle_bf16_to_f64(x[(r0 + i) * ld + c]);
+      halo_oracle_fwht(col, blk);
+      for (int64_t i = 0; i < blk; ++i) v[(r0 + i) * cols + c] = col[i];
+    }
+  }
+  free(col);
+}
+
 /* ------------------------------------------------------------------------ */
 /* OCP FP8 E4M3 ("fn": no infinities, max finite 448).  Sign, 4 exponent    */
 /* bits with bias 7, 3 mantissa bits.  Exponent field 0 holds subnormals    */
@@ -231,6 +260,61 @@ void halo_oracle_quantize(const double* v, int64_t rows, int64_t cols, int axis,
         codes[idx] = (uint8_t)(int8_t)q;
       } else {
         codes[idx] = halo_oracle_e4m3_encode(t);
+      }
+    }
+  }
+}
+
+/* Stochastic-rounding variant of the quantiser [QWHA page sec. 5: random
+ * rounding reduces the bias of quantisation, floor(x) + (rand < x - floor(x))].
+ * Same scale as above; the code of element idx rounds t = v / s to one of its
+ * two grid neighbours lo <= t < hi, taking hi when u < (t - lo) / (hi - lo),
+ * with u = rand[idx] / 65536 (16 caller-supplied random bits per element).
+ * INT8 grid: the integers, clamped to +-127.  E4M3 grid: the E4M3 values,
+ * saturating at 448 (|t| >= 448 gives +-448).  rand[] has the layout of v. */
+static double e4m3_quantum(double a) {
+  if (a < ldexp(1.0, -6)) return ldexp(1.0, -9);
+  int ex;
+  frexp(a, &ex);
+  return ldexp(1.0, (ex - 1) - 3);
+}
+
+void halo_oracle_quantize_stochastic(const double* v, int64_t rows, int64_t cols, int axis, int qtype,
+                                     const uint16_t* rand, uint8_t* codes, float* scales, double* t_out) {
+  const double qmax = (qtype == 0) ? 127.0 : 448.0;
+  const int64_t groups = (axis == 0) ? rows : cols;
+  const int64_t len = (axis == 0) ? cols : rows;
+  for (int64_t g = 0; g < groups; ++g) {
+    double amax = 0.0;
+    for (int64_t i = 0; i < len; ++i) {
+      int64_t idx = (axis == 0) ? g * cols + i : i * cols + g;
+      double a = fabs(v[idx]);
+      if (a > amax) amax = a;
+    }
+    float s = (float)(amax / qmax);
+    scales[g] = s;
+    for (int64_t i = 0; i < len; ++i) {
+      int64_t idx = (axis == 0) ? g * cols + i : i * cols + g;
+      double t = (s == 0.0f) ? 0.0 : v[idx] / (double)s;
+      double u = (double)rand[idx] / 65536.0;
+      if (t_out) t_out[idx] = t;
+      if (qtype == 0) {
+        double lo = floor(t);
+        double q = (u < t - lo) ? lo + 1.0 : lo;
+        if (q > 127.0) q = 127.0;
+        if (q < -127.0) q = -127.0;
+        codes[idx] = (uint8_t)(int8_t)q;
+      } else {
+        double a = fabs(t);
+        double mag;
+        if (a >= 448.0) {
+          mag = 448.0;
+        } else {
+          double quantum = e4m3_quantum(a);
+          double lo = floor(a / quantum) * quantum;
+          mag = (u < (a - lo) / quantum) ? lo + quantum : lo;
+        }
+        codes[idx] = halo_oracle_e4m3_encode(signbit(t) ? -mag : mag);
       }
     }
   }

@@ -350,3 +350,92 @@ def test_composition_of_rotated_qgemm_parts():
     aq, sa, bq, sb = oracle.rotated_qgemm_parts(x, True, w, True, 128, oracle.INT8)
     y = oracle.dequant(oracle.gemm_i8(aq, bq).astype(np.float64), sa, sb)
     np.testing.assert_array_equal(y, oracle.linear_fwd(x, w, 128, oracle.INT8))
+
+
+# ------------------------------------------------------------- random-sign rotation
+def _signs(n, seed):
+    rng = np.random.default_rng(seed)
+    return np.where(rng.random(n) < 0.5, -1, 1).astype(np.int8)
+
+
+def test_signed_rotation_all_plus_is_plain_rotation():
+    rng = np.random.default_rng(31)
+    x = torch.from_numpy(rng.standard_normal((8, 512)).astype(np.float32)).to(torch.bfloat16)
+    ones = np.ones(512, dtype=np.int8)
+    np.testing.assert_array_equal(oracle.rotate_signed(x, 128, 1, ones), oracle.rotate(x, 128, 1))
+    np.testing.assert_array_equal(oracle.rotate_signed(x.t().contiguous(), 128, 0, ones),
+                                  oracle.rotate(x.t().contiguous(), 128, 0))
+
+
+def test_signed_rotation_equals_dense_h_times_diag():
+    rng = np.random.default_rng(32)
+    x = torch.from_numpy(rng.standard_normal((5, 256)).astype(np.float32)).to(torch.bfloat16)
+    s = _signs(256, 1)
+    hb = _sylvester_block(128) / np.sqrt(128)
+    dense = scipy.linalg.block_diag(hb, hb) @ np.diag(s.astype(np.float64))
+    np.testing.assert_allclose(oracle.rotate_signed(x, 128, 1, s), x.double().numpy() @ dense.T, atol=1e-11)
+    got0 = oracle.rotate_signed(x.t().contiguous(), 128, 0, s)
+    np.testing.assert_allclose(got0, oracle.rotate_signed(x, 128, 1, s).T, atol=1e-12)
+
+
+def test_signed_rotation_keeps_the_product_only_with_matching_signs():
+    rng = np.random.default_rng(33)
+    x = torch.from_numpy(rng.standard_normal((16, 384)).astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy(rng.standard_normal((12, 384)).astype(np.float32)).to(torch.bfloat16)
+    s = _signs(384, 2)
+    ref = x.double().numpy() @ w.double().numpy().T
+    same = oracle.rotate_signed(x, 128, 1, s) @ oracle.rotate_signed(w, 128, 1, s).T
+    np.testing.assert_allclose(same, ref, atol=1e-10 * np.max(np.abs(ref)))
+    other = oracle.rotate_signed(x, 128, 1, s) @ oracle.rotate_signed(w, 128, 1, _signs(384, 3)).T
+    assert np.max(np.abs(other - ref)) > 0.1 * np.max(np.abs(ref))
+
+
+# ----------------------------------------------------------- stochastic rounding
+def test_golden_stochastic_quantisation():
+    for qt, row, bits, codes in _rows("quantize_stochastic_worked.txt"):
+        v = np.array([[float(t) for t in row.split()]])
+        rb = np.array([[int(b) for b in bits.split()]], dtype=np.uint16)
+        qtype = oracle.INT8 if qt == "int8" else oracle.E4M3
+        q, s, _ = oracle.quantize_stochastic(v, 0, qtype, rb)
+        assert s[0] == 1.0
+        if qtype == oracle.INT8:
+            np.testing.assert_array_equal(q.view(np.int8)[0], [int(c) for c in codes.split()])
+        else:
+            np.testing.assert_array_equal(q[0], [int(c, 16) for c in codes.split()])
+
+
+def test_stochastic_codes_are_grid_neighbours_with_rne_scales():
+    rng = np.random.default_rng(34)
+    v = rng.standard_normal((20, 256)) * 3
+    rb = rng.integers(0, 65536, size=v.shape).astype(np.uint16)
+    for qt in (oracle.INT8, oracle.E4M3):
+        q, s, t = oracle.quantize_stochastic(v, 0, qt, rb)
+        _, s_rne, t_rne = oracle.quantize(v, 0, qt)
+        np.testing.assert_array_equal(s, s_rne)
+        np.testing.assert_array_equal(t, t_rne)
+        if qt == oracle.INT8:
+            qi = q.view(np.int8).astype(np.float64)
+            assert np.all((qi == np.floor(t)) | (qi == np.floor(t) + 1) | (np.abs(qi) == 127))
+        else:
+            d = oracle.e4m3_decode(q)
+            a = np.abs(t)
+            quantum = np.where(a < 2.0**-6, 2.0**-9, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-300))) - 3))
+            lo = np.floor(a / quantum) * quantum
+            assert np.all((np.abs(d) == lo) | (np.abs(d) == lo + quantum) | (np.abs(d) == 448))
+            assert np.all((d == 0) | (np.sign(d) == np.sign(t)))
+
+
+def test_stochastic_rounding_is_unbiased():
+    """E[q] = t up to the 2^-16 resolution of the random bits."""
+    rng = np.random.default_rng(35)
+    row = np.concatenate([[127.0], rng.uniform(-120, 120, 63)])
+    trials = 4000
+    v = np.tile(row, (trials, 1))
+    rb = rng.integers(0, 65536, size=v.shape).astype(np.uint16)
+    q, s, t = oracle.quantize_stochastic(v, 0, oracle.INT8, rb)
+    mean = q.view(np.int8).astype(np.float64).mean(axis=0)
+    # each code is a Bernoulli step of 1: sd <= 0.5 / sqrt(trials)
+    assert np.all(np.abs(mean - t[0]) <= 5 * 0.5 / np.sqrt(trials) + 2.0**-16)
+    # round to nearest is biased on the same values; stochastic is not
+    q_rne, _, _ = oracle.quantize(v[:1], 0, oracle.INT8)
+    assert np.mean(np.abs(q_rne.view(np.int8)[0] - t[0])) > 4 * np.mean(np.abs(mean - t[0]))
