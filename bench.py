@@ -486,6 +486,35 @@ def measure_rotq_shapes(repeats: int = 10):
                 out.append({"direction": name, "shape": [r, c], "qtype": "int8" if qt == 0 else "e4m3",
                             "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
             del x, q, sc
+    # The variants (halo_hadamard_quantize_ex): random signs along the rotated
+    # dimension and stochastic rounding from 16 random bits per element (which
+    # add 2 B per element of input traffic).
+    g = torch.Generator(device="cuda").manual_seed(7)
+    for name, shapes in ROTQ_SHAPES.items():
+        axis = halo.HALO_AXIS_COLS if name == "along_contiguous_dim" else halo.HALO_AXIS_ROWS
+        for r, c in shapes[:2] + shapes[-1:]:
+            x = inputs.activations(r, c, seed=1, device="cuda")
+            signs = (torch.randint(0, 2, (c if axis == halo.HALO_AXIS_COLS else r,), device="cuda", generator=g,
+                                   dtype=torch.int8) * 2 - 1).to(torch.int8)
+            rand = torch.randint(0, 65536, (r, c), device="cuda", generator=g, dtype=torch.int32).to(torch.uint16)
+            for variant, sg, rb in (("signs", signs, None), ("stochastic", None, rand), ("signs+stochastic", signs, rand)):
+                q, sc = halo.halo_hadamard_quantize_ex(x, axis, BLK, halo.HALO_Q_INT8, signs=sg, rand_bits=rb)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(repeats):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    halo.halo_hadamard_quantize_ex(x, axis, BLK, halo.HALO_Q_INT8, signs=sg, rand_bits=rb, q_out=q,
+                                                   scales_out=sc)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                ms = sorted(ts)[len(ts) // 2]
+                nbytes = (3 + (2 if rb is not None else 0)) * x.numel() + 4 * sc.numel() + (sg.numel() if sg is not None else 0)
+                out.append({"direction": name, "shape": [r, c], "qtype": "int8", "variant": variant,
+                            "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
+            del x, q, sc, rand, signs
     return {"measure": "rotate+quantise per shape", "block": BLK, "results": out}
 
 

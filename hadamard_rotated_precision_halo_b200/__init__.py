@@ -39,6 +39,7 @@ HALO_MAJOR_MN = 1
 
 EXPORTS = (
     "halo_hadamard_quantize",
+    "halo_hadamard_quantize_ex",
     "halo_qgemm",
     "halo_workspace_size",
     "halo_linear_fwd",
@@ -76,6 +77,8 @@ def lib():
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     L.halo_hadamard_quantize.argtypes = [P, I64, I64, I64, I, I, I, P, I64, P, P]
     L.halo_hadamard_quantize.restype = I
+    L.halo_hadamard_quantize_ex.argtypes = [P, I64, I64, I64, I, I, I, P, P, I64, P, I64, P, P]
+    L.halo_hadamard_quantize_ex.restype = I
     L.halo_qgemm.argtypes = [P, P, I, I64, P, P, I, I64, I64, I64, I64, I, P, I, I64, P]
     L.halo_qgemm.restype = I
     L.halo_workspace_size.argtypes = [I64, I64, I64, I]
@@ -140,6 +143,24 @@ def halo_hadamard_quantize(x: torch.Tensor, axis: int, blk: int, qtype: int, q_o
     st = lib().halo_hadamard_quantize(_ptr(x), rows, cols, x.stride(0), axis, blk, qtype, _ptr(q_out),
                                       q_out.stride(0), _ptr(scales_out), _stream(stream))
     _check(st, "halo_hadamard_quantize")
+    return q_out, scales_out
+
+
+def halo_hadamard_quantize_ex(x: torch.Tensor, axis: int, blk: int, qtype: int, signs=None, rand_bits=None,
+                              q_out=None, scales_out=None, stream=None):
+    """halo_hadamard_quantize with optional +-1 signs along the rotated dimension
+    (int8 tensor) and optional per-element random bits for stochastic rounding
+    (uint16 stored as int16/uint16 tensor of x's shape)."""
+    rows, cols = x.shape
+    if q_out is None:
+        q_out = torch.empty((rows, cols), dtype=_code_dtype(qtype), device=x.device)
+    if scales_out is None:
+        scales_out = torch.empty(rows if axis == HALO_AXIS_COLS else cols, dtype=torch.float32, device=x.device)
+    ld_rand = rand_bits.stride(0) if rand_bits is not None else 0
+    st = lib().halo_hadamard_quantize_ex(_ptr(x), rows, cols, x.stride(0), axis, blk, qtype, _ptr(signs),
+                                         _ptr(rand_bits), ld_rand, _ptr(q_out), q_out.stride(0), _ptr(scales_out),
+                                         _stream(stream))
+    _check(st, "halo_hadamard_quantize_ex")
     return q_out, scales_out
 
 

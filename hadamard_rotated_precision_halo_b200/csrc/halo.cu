@@ -65,20 +65,39 @@ cudaError_t set_smem_attr(K kernel, int optin) {
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
+typedef void (*RowsKernel)(const CUtensorMap, const CUtensorMap, RotqRowsParams);
 typedef void (*Cols1Kernel)(const CUtensorMap, const CUtensorMap, RotqCols1Params);
+typedef void (*Cols2Kernel)(const CUtensorMap, const CUtensorMap, RotqColsParams);
 
-template <int QT>
+// `ext`: the instantiation that reads the variants' optional inputs (signs,
+// random bits); the plain path is compiled without them.
+RowsKernel rows_kernel(int blk, int qtype, bool ext) {
+  if (blk == 128) {
+    if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<128, 0, 1> : rotq_rows_kernel<128, 0, 0>;
+    return ext ? rotq_rows_kernel<128, 1, 1> : rotq_rows_kernel<128, 1, 0>;
+  }
+  if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<256, 0, 1> : rotq_rows_kernel<256, 0, 0>;
+  return ext ? rotq_rows_kernel<256, 1, 1> : rotq_rows_kernel<256, 1, 0>;
+}
+
+template <int QT, int EXT>
 Cols1Kernel cols_1pass_for(int nw) {
   switch (nw) {
-    case 1: return rotq_cols_1pass_kernel<QT, 1>;
-    case 2: return rotq_cols_1pass_kernel<QT, 2>;
-    case 3: return rotq_cols_1pass_kernel<QT, 3>;
-    default: return rotq_cols_1pass_kernel<QT, 4>;
+    case 1: return rotq_cols_1pass_kernel<QT, 1, EXT>;
+    case 2: return rotq_cols_1pass_kernel<QT, 2, EXT>;
+    case 3: return rotq_cols_1pass_kernel<QT, 3, EXT>;
+    default: return rotq_cols_1pass_kernel<QT, 4, EXT>;
   }
 }
 
-Cols1Kernel cols_1pass_kernel(int qtype, int nw) {
-  return qtype == HALO_Q_INT8 ? cols_1pass_for<0>(nw) : cols_1pass_for<1>(nw);
+Cols1Kernel cols_1pass_kernel(int qtype, int nw, bool ext) {
+  if (qtype == HALO_Q_INT8) return ext ? cols_1pass_for<0, 1>(nw) : cols_1pass_for<0, 0>(nw);
+  return ext ? cols_1pass_for<1, 1>(nw) : cols_1pass_for<1, 0>(nw);
+}
+
+Cols2Kernel cols_2pass_kernel(int qtype, bool ext) {
+  if (qtype == HALO_Q_INT8) return ext ? rotq_cols_kernel<0, 1> : rotq_cols_kernel<0, 0>;
+  return ext ? rotq_cols_kernel<1, 1> : rotq_cols_kernel<1, 0>;
 }
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
@@ -110,16 +129,16 @@ halo_status_t device_setup(int* dev_out) {
     }
     int optin = 0;
     HALO_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 0>, optin));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<128, 1>, optin));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 0>, optin));
-    HALO_CUDA(set_smem_attr(rotq_rows_kernel<256, 1>, optin));
-    HALO_CUDA(set_smem_attr(rotq_cols_kernel<0>, optin));
-    HALO_CUDA(set_smem_attr(rotq_cols_kernel<1>, optin));
-    for (int nw = 1; nw <= 4; ++nw) {
+    for (int e = 0; e < 2; ++e) {
       for (int qt = 0; qt < 2; ++qt) {
-        HALO_CUDA(set_smem_attr(cols_1pass_kernel(qt, nw), optin));
-        HALO_CUDA(cudaFuncSetAttribute(cols_1pass_kernel(qt, nw), cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        HALO_CUDA(set_smem_attr(rows_kernel(128, qt, e), optin));
+        HALO_CUDA(set_smem_attr(rows_kernel(256, qt, e), optin));
+        HALO_CUDA(set_smem_attr(cols_2pass_kernel(qt, e), optin));
+        for (int nw = 1; nw <= 4; ++nw) {
+          HALO_CUDA(set_smem_attr(cols_1pass_kernel(qt, nw, e), optin));
+          HALO_CUDA(cudaFuncSetAttribute(cols_1pass_kernel(qt, nw, e),
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        }
       }
     }
     HALO_CUDA(set_smem_attr(qgemm_kernel<0>, optin));
@@ -194,7 +213,8 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
 
 // ------------------------------------------------------------------------ rotq launches
 halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
-                               void* q, int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
+                               void* q, int64_t ld_q, float* scales, const RotqExtras& ex, bool ext,
+                               cudaStream_t stream, int dev) {
   const int nb = static_cast<int>(cols / 128);
   // A row group of ceil(nb / 32) warps owns one row at a time; 4 warps per
   // CTA when a group fits in 4, else one group per CTA (up to 8 warps).
@@ -229,12 +249,9 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   p.groups = groups;
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(static_cast<double>(blk))));
+  p.ex = ex;
 
-  void (*kern)(const CUtensorMap, const CUtensorMap, RotqRowsParams) = nullptr;
-  if (blk == 128)
-    kern = qtype == HALO_Q_INT8 ? rotq_rows_kernel<128, 0> : rotq_rows_kernel<128, 1>;
-  else
-    kern = qtype == HALO_Q_INT8 ? rotq_rows_kernel<256, 0> : rotq_rows_kernel<256, 1>;
+  RowsKernel kern = rows_kernel(blk, qtype, ext);
   int per_sm = 0;
   HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
   if (per_sm < 1) per_sm = 1;
@@ -248,7 +265,8 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
 // Single pass when the 128-row blocks of a column strip split evenly over a
 // cluster of at most 16 CTAs with at most 4 warps each (R <= 8192 rows).
 halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
-                                     int64_t ld_q, float* scales, cudaStream_t stream, int nw, int cl, int dev) {
+                                     int64_t ld_q, float* scales, const RotqExtras& ex, bool ext,
+                                     cudaStream_t stream, int nw, int cl, int dev) {
   const int strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
   CUtensorMap tm_x, tm_q;
   {
@@ -273,7 +291,8 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
   p.strips = strips;
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
-  Cols1Kernel kern = cols_1pass_kernel(qtype, nw);
+  p.ex = ex;
+  Cols1Kernel kern = cols_1pass_kernel(qtype, nw, ext);
 
   // Persistent: as many clusters as fit at once (each loops over strips).
   Launch L(dim3(cl, 1, 1), dim3(32 * nw), static_cast<size_t>(nw) * (2 * kColsInBytes + kColsOutBytes) + 128,
@@ -289,12 +308,14 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
 }
 
 halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
-                               int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
+                               int64_t ld_q, float* scales, const RotqExtras& ex, bool ext, cudaStream_t stream,
+                               int dev) {
   const int nblocks = static_cast<int>(rows / 128);
   // Most warps per CTA (up to 4) with at most 16 CTAs per cluster.
   for (int nw = 4; nw >= 1; --nw) {
     if (nblocks % nw == 0 && nblocks / nw <= 16)
-      return launch_rotq_cols_1pass(x, rows, cols, ld_x, qtype, q, ld_q, scales, stream, nw, nblocks / nw, dev);
+      return launch_rotq_cols_1pass(x, rows, cols, ld_x, qtype, q, ld_q, scales, ex, ext, stream, nw, nblocks / nw,
+                                    dev);
   }
   // Taller matrices: the two-pass kernel (column maxima first, then codes).
   int cl = 8;
@@ -326,13 +347,11 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
   p.warps = warps;
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  p.ex = ex;
   const size_t smem = static_cast<size_t>(warps) * (kColsStages * kColsInBytes + 2 * kColsOutBytes) + 128;
 
   Launch L(dim3(cl, strips, 1), dim3(32 * warps), smem, stream, cl);
-  if (qtype == HALO_Q_INT8)
-    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, rotq_cols_kernel<0>, tm_x, tm_q, p));
-  else
-    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, rotq_cols_kernel<1>, tm_x, tm_q, p));
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, cols_2pass_kernel(qtype, ext), tm_x, tm_q, p));
   return HALO_OK;
 }
 
@@ -441,6 +460,15 @@ halo_status_t check_hadamard_quantize(const void* x, int64_t rows, int64_t cols,
   return HALO_OK;
 }
 
+halo_status_t check_extras(const int8_t* signs, const uint16_t* rand_bits, int64_t ld_rand, int64_t cols) {
+  if (signs && !aligned16(signs)) return HALO_ERR_ALIGN;
+  if (rand_bits) {
+    if (ld_rand < cols) return HALO_ERR_SHAPE;
+    if (!aligned16(rand_bits) || (ld_rand * 2) % 16 != 0) return HALO_ERR_ALIGN;
+  }
+  return HALO_OK;
+}
+
 halo_status_t check_qgemm(const void* a, const float* sa, int a_major, int64_t ld_a, const void* b,
                           const float* sb, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k, int qtype,
                           const void* c, int otype, int64_t ld_c) {
@@ -538,17 +566,32 @@ size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which) {
   return ws_layout(m, n, k, which).total;
 }
 
-halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int axis,
-                                     int blk, int qtype, void* q_out, int64_t ld_q, float* scales_out,
-                                     void* stream) {
+halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int axis,
+                                        int blk, int qtype, const int8_t* signs, const uint16_t* rand_bits,
+                                        int64_t ld_rand, void* q_out, int64_t ld_q, float* scales_out,
+                                        void* stream) {
   halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, axis, blk, qtype, q_out, ld_q, scales_out);
   if (st != HALO_OK) return st;
+  if ((st = check_extras(signs, rand_bits, ld_rand, cols)) != HALO_OK) return st;
   int dev = 0;
   st = device_setup(&dev);
   if (st != HALO_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (axis == HALO_AXIS_COLS) return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, qtype, q_out, ld_q, scales_out, s, dev);
-  return launch_rotq_cols(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, s, dev);
+  RotqExtras ex;
+  ex.signs = signs;
+  ex.rand = rand_bits;
+  ex.ld_rand = rand_bits ? ld_rand : 0;
+  const bool ext = signs != nullptr || rand_bits != nullptr;
+  if (axis == HALO_AXIS_COLS)
+    return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, qtype, q_out, ld_q, scales_out, ex, ext, s, dev);
+  return launch_rotq_cols(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, ex, ext, s, dev);
+}
+
+halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int axis,
+                                     int blk, int qtype, void* q_out, int64_t ld_q, float* scales_out,
+                                     void* stream) {
+  return halo_hadamard_quantize_ex(x_bf16, rows, cols, ld_x, axis, blk, qtype, nullptr, nullptr, 0, q_out, ld_q,
+                                   scales_out, stream);
 }
 
 halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,

@@ -125,6 +125,58 @@ __device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
+// Optional inputs of the rotate+quantise variants (used when a kernel is
+// instantiated with EXT = 1):
+//   signs  +-1 per position along the rotated dimension (random-sign
+//          rotation H (D x)); only the sign bit is used.  nullptr: none.
+//   rand   16 random bits per element, layout [rows, cols] with row stride
+//          ld_rand: stochastic rounding with u = rand / 65536.  nullptr:
+//          round to nearest even.
+struct RotqExtras {
+  const int8_t* signs;
+  const uint16_t* rand;
+  int64_t ld_rand;
+};
+
+// bf16x2 sign-flip mask from two sign bytes of a 4-byte group (pair 0: bytes
+// 0, 1; pair 1: bytes 2, 3): bit 15 and bit 31 take the bytes' sign bits.
+__device__ __forceinline__ uint32_t sign_mask_pair(uint32_t s4, int pair) {
+  return __byte_perm(s4, 0u, pair ? 0x3424 : 0x1404) & 0x80008000u;
+}
+
+// bf16x2 sign-flip mask for both halves from sign byte `b` (0..3) of s4.
+__device__ __forceinline__ uint32_t sign_mask_row(uint32_t s4, int b) {
+  const uint32_t sel = (static_cast<uint32_t>(b) << 12) | (4u << 8) | (static_cast<uint32_t>(b) << 4) | 4u;
+  return __byte_perm(s4, 0u, sel) & 0x80008000u;
+}
+
+// Stochastic rounding onto the INT8 grid: the upper neighbour of t when
+// uu < t - floor(t); clamped to +-127; the code in the low byte.
+__device__ __forceinline__ uint32_t q_int8_sr(float t, float uu) {
+  const float lo = floorf(t);
+  float q = (uu < t - lo) ? lo + 1.f : lo;
+  q = fminf(fmaxf(q, -127.f), 127.f);
+  return static_cast<uint32_t>(__float2int_rn(q)) & 0xFFu;
+}
+
+// Stochastic rounding onto the E4M3 grid: the signed grid value to encode.
+// Grid spacing 2^-9 below 2^-6, else 2^(floor(log2|t|) - 3); |t| >= 448 gives 448.
+__device__ __forceinline__ float e4m3_sr_value(float t, float uu) {
+  const float a = fabsf(t);
+  float mag;
+  if (a >= 448.f) {
+    mag = 448.f;
+  } else {
+    const float quantum =
+        a < 0.015625f ? 0.001953125f : __uint_as_float(((__float_as_uint(a) >> 23) - 3u) << 23);
+    const float lo = floorf(__fdiv_rn(a, quantum)) * quantum;  // exact: quantum is a power of two
+    mag = (uu < __fdiv_rn(a - lo, quantum)) ? lo + quantum : lo;
+  }
+  return copysignf(mag, t);
+}
+
+__device__ __forceinline__ float rand_unit(uint32_t bits16) { return static_cast<float>(bits16) * (1.f / 65536.f); }
+
 // ------------------------------------------------------------------------------------------
 // rotq_rows: one thread owns one 128-element chunk of one row.  A row is
 // handled by a "row group" of G = ceil(nb / 32) warps (one warp when the row
@@ -146,6 +198,7 @@ struct RotqRowsParams {
   int groups;    // row groups per CTA
   float qmax;
   float scale_mult;  // 1 / (qmax * sqrt(blk))
+  RotqExtras ex;     // EXT = 1 only
 };
 
 // Shared-memory bytes of one row group: 2 input stages and one code tile.
@@ -160,7 +213,7 @@ __device__ __forceinline__ void group_sync(int gw, int grp) {
     named_bar_sync(1 + grp, gw * 32);
 }
 
-template <int BLK, int QT>
+template <int BLK, int QT, int EXT>
 __global__ void __launch_bounds__(256)
     rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                      RotqRowsParams p) {
@@ -219,9 +272,20 @@ __global__ void __launch_bounds__(256)
     float2 v[64];
     if (is_active && !dead) {
       const uint4* src = reinterpret_cast<const uint4*>(g_in + st * rows_group_in_bytes(gw) + chunk * kRowsInSlot);
+      const uint4* sgn = reinterpret_cast<const uint4*>(p.ex.signs + static_cast<int64_t>(chunk) * 128);
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        const uint4 raw = src[k];
+        uint4 raw = src[k];
+        if (EXT && p.ex.signs != nullptr) {
+          // elements 8k .. 8k+7: sign bytes 8k .. 8k+7 = half of sign vector k/2
+          const uint4 sv = __ldg(sgn + k / 2);
+          const uint32_t s01 = (k & 1) ? sv.z : sv.x;
+          const uint32_t s23 = (k & 1) ? sv.w : sv.y;
+          raw.x ^= sign_mask_pair(s01, 0);
+          raw.y ^= sign_mask_pair(s01, 1);
+          raw.z ^= sign_mask_pair(s23, 0);
+          raw.w ^= sign_mask_pair(s23, 1);
+        }
         v[4 * k + 0] = bf16x2_to_f2(raw.x);
         v[4 * k + 1] = bf16x2_to_f2(raw.y);
         v[4 * k + 2] = bf16x2_to_f2(raw.z);
@@ -263,6 +327,9 @@ __global__ void __launch_bounds__(256)
     if (chunk == 0) p.scales[row] = row_amax * p.scale_mult;
     if (is_active) {
       uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
+      const uint4* rnd = EXT ? reinterpret_cast<const uint4*>(p.ex.rand + row * p.ex.ld_rand +
+                                                                static_cast<int64_t>(chunk) * 128)
+                             : nullptr;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         uint32_t w[4];
@@ -270,6 +337,22 @@ __global__ void __launch_bounds__(256)
         for (int j = 0; j < 4; ++j) {
           const float2 a = v[8 * k + 2 * j];
           const float2 b = v[8 * k + 2 * j + 1];
+          if (EXT && p.ex.rand != nullptr) {
+            // elements 16k + 4j .. +3: random halves 4(j%2) .. +3 of vector 2k + j/2
+            const uint4 rv = __ldg(rnd + 2 * k + j / 2);
+            const uint32_t r01 = (j & 1) ? rv.z : rv.x;
+            const uint32_t r23 = (j & 1) ? rv.w : rv.y;
+            const float u0 = rand_unit(r01 & 0xFFFFu), u1 = rand_unit(r01 >> 16);
+            const float u2 = rand_unit(r23 & 0xFFFFu), u3 = rand_unit(r23 >> 16);
+            if (QT == 0) {
+              w[j] = pack4_int8(q_int8_sr(a.x * r, u0), q_int8_sr(a.y * r, u1), q_int8_sr(b.x * r, u2),
+                                q_int8_sr(b.y * r, u3));
+            } else {
+              w[j] = e4m3x2_bits(e4m3_sr_value(a.x * r, u0), e4m3_sr_value(a.y * r, u1)) |
+                     (e4m3x2_bits(e4m3_sr_value(b.x * r, u2), e4m3_sr_value(b.y * r, u3)) << 16);
+            }
+            continue;
+          }
           if (QT == 0) {
             w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r),
                               q_int8_bits(b.y, r));
@@ -300,12 +383,22 @@ constexpr int kColsStages = 2;
 // both rows of every pair forms the bottom butterfly stage on the way in
 // (h = 0 keeps the sum, h = 1 the difference); the other six stages run on
 // the lane's own rows.
-__device__ __forceinline__ void cols_load_fwht(const uint32_t* blkw, int pcol, int h, float2 (&v)[64]) {
+// `row_signs` (EXT only): the +-1 signs of the block's 128 rows, or nullptr.
+template <int EXT = 0>
+__device__ __forceinline__ void cols_load_fwht(const uint32_t* blkw, int pcol, int h, float2 (&v)[64],
+                                               const int8_t* row_signs = nullptr) {
   const float sg = h ? -1.f : 1.f;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
-    const float2 a = bf16x2_to_f2(blkw[(2 * i) * 16 + pcol]);
-    const float2 b = bf16x2_to_f2(blkw[(2 * i + 1) * 16 + pcol]);
+    uint32_t wa = blkw[(2 * i) * 16 + pcol];
+    uint32_t wb = blkw[(2 * i + 1) * 16 + pcol];
+    if (EXT && row_signs != nullptr) {
+      const uint32_t s4 = __ldg(reinterpret_cast<const uint32_t*>(row_signs) + i / 2);  // rows 4(i/2) .. +3
+      wa ^= sign_mask_row(s4, 2 * (i & 1));
+      wb ^= sign_mask_row(s4, 2 * (i & 1) + 1);
+    }
+    const float2 a = bf16x2_to_f2(wa);
+    const float2 b = bf16x2_to_f2(wb);
     v[i] = __ffma2_rn(b, make_float2(sg, sg), a);
   }
 }
@@ -325,13 +418,25 @@ __device__ __forceinline__ void cols_fwht_rest(float2 (&v)[64]) {
 }
 
 // Codes of the lane's 64 rows x 2 columns into a [128][32]-byte tile.
-template <int QT>
+// `rnd` (EXT only): random bits of this lane's two columns in the block's
+// first row (stride ld_rand between rows), or nullptr for round to nearest.
+template <int QT, int EXT = 0>
 __device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
-                                                 int h) {
+                                                 int h, const uint16_t* rnd = nullptr, int64_t ld_rand = 0) {
   uint16_t* outw = reinterpret_cast<uint16_t*>(tile);
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     uint32_t code;
+    if (EXT && rnd != nullptr) {
+      const uint32_t rb = __ldg(reinterpret_cast<const uint32_t*>(rnd + (2 * i + h) * ld_rand));
+      const float u0 = rand_unit(rb & 0xFFFFu), u1 = rand_unit(rb >> 16);
+      if (QT == 0)
+        code = __byte_perm(q_int8_sr(v[i].x * r0, u0), q_int8_sr(v[i].y * r1, u1), 0x0040) & 0xFFFFu;
+      else
+        code = e4m3x2_bits(e4m3_sr_value(v[i].x * r0, u0), e4m3_sr_value(v[i].y * r1, u1));
+      outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
+      continue;
+    }
     if (QT == 0) {
       code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
     } else {
@@ -348,9 +453,10 @@ struct RotqColsParams {
   int warps;       // warps per CTA
   float qmax;
   float scale_mult;  // 1 / (qmax * sqrt(128))
+  RotqExtras ex;     // EXT = 1 only
 };
 
-template <int QT>
+template <int QT, int EXT>
 __global__ void __launch_bounds__(128)
     rotq_cols_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                      RotqColsParams p) {
@@ -416,7 +522,10 @@ __global__ void __launch_bounds__(128)
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
-    cols_load_fwht(blkw, pcol, h, v);
+    {
+      const int b = first + step * j;
+      cols_load_fwht<EXT>(blkw, pcol, h, v, EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(b) * 128 : nullptr);
+    }
     __syncwarp();
     if (lane == 0 && j + kColsStages < nseq) issue(j + kColsStages);
     cols_fwht_rest(v);
@@ -456,7 +565,8 @@ __global__ void __launch_bounds__(128)
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
-    cols_load_fwht(blkw, pcol, h, v);
+    const int bq = first + step * (j - nmine);
+    cols_load_fwht<EXT>(blkw, pcol, h, v, EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(bq) * 128 : nullptr);
     __syncwarp();
     if (lane == 0) {
       if (j + kColsStages < nseq) issue(j + kColsStages);
@@ -464,12 +574,17 @@ __global__ void __launch_bounds__(128)
     }
     cols_fwht_rest(v);
     __syncwarp();
-    cols_write_codes<QT>(s_out + ob * kColsOutBytes, v, r0, r1, pcol, h);
+    {
+      const bool col_ok = c0 + 2 * pcol < p.cols;
+      const uint16_t* rnd = EXT && p.ex.rand && col_ok
+                                ? p.ex.rand + static_cast<int64_t>(bq) * 128 * p.ex.ld_rand + c0 + 2 * pcol
+                                : nullptr;
+      cols_write_codes<QT, EXT>(s_out + ob * kColsOutBytes, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      const int b = first + step * (j - nmine);
-      tma_store_2d(&tm_q, s_out + ob * kColsOutBytes, c0, b * 128);
+      tma_store_2d(&tm_q, s_out + ob * kColsOutBytes, c0, bq * 128);
       bulk_commit();
     }
   }
@@ -501,11 +616,12 @@ struct RotqCols1Params {
   int strips;  // ceil(cols / 32)
   float qmax;
   float scale_mult;  // 1 / (qmax * sqrt(128))
+  RotqExtras ex;     // EXT = 1 only
 };
 
 enum : unsigned int { kSiteRotqCols1Load = 0x202, kSiteRotqCols1Reduce = 0x203 };
 
-template <int QT, int NW>
+template <int QT, int NW, int EXT>
 __global__ void __launch_bounds__(NW * 32)
     rotq_cols_1pass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                            RotqCols1Params p) {
@@ -572,7 +688,8 @@ __global__ void __launch_bounds__(NW * 32)
       dead = __any_sync(0xffffffffu, !ok);
     }
     if (!dead) {
-      cols_load_fwht(reinterpret_cast<const uint32_t*>(s_in + par * kColsInBytes), pcol, h, v);
+      cols_load_fwht<EXT>(reinterpret_cast<const uint32_t*>(s_in + par * kColsInBytes), pcol, h, v,
+                          EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(blk) * 128 : nullptr);
     } else {
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
@@ -616,7 +733,13 @@ __global__ void __launch_bounds__(NW * 32)
     }
     if (lane == 0) bulk_wait_read<0>();  // the previous strip's store has read the code tile
     __syncwarp();
-    cols_write_codes<QT>(s_out, v, r0, r1, pcol, h);
+    {
+      const bool col_ok = c0 + 2 * pcol < p.cols;
+      const uint16_t* rnd = EXT && p.ex.rand && col_ok
+                                ? p.ex.rand + static_cast<int64_t>(blk) * 128 * p.ex.ld_rand + c0 + 2 * pcol
+                                : nullptr;
+      cols_write_codes<QT, EXT>(s_out, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {

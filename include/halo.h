@@ -100,6 +100,30 @@ halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t c
                                      float* scales_out, void* stream);
 
 /*
+ * halo_hadamard_quantize with the two variants of the rotation and rounding:
+ *   signs      NULL, or int8 +1 / -1 (only the sign bit is read) for every
+ *              position along the rotated dimension (`cols` entries for
+ *              HALO_AXIS_COLS, `rows` for HALO_AXIS_ROWS), 16-byte aligned:
+ *              random-sign rotation, each block becomes H_blk D x / sqrt(blk)
+ *              with D = diag(signs).  Both operands of a GEMM must use the
+ *              same signs along the contraction dimension; the product is
+ *              then unchanged, since (H D)^T (H D) = I.  Seeded random signs
+ *              shared by all workers: HALO blog page, sec. 4.2.
+ *   rand_bits  NULL (round half to even), or 16 random bits per element,
+ *              layout [rows, cols] with row stride ld_rand elements (16-byte
+ *              aligned base, ld_rand * 2 a multiple of 16): stochastic
+ *              rounding.  With u = rand_bits / 65536, t = Xrot / s rounds to
+ *              its upper grid neighbour when u < (t - lo) / (hi - lo), else
+ *              to its lower one (INT8 grid clamped to +-127; E4M3 grid
+ *              saturating at 448).  QWHA page, sec. 5 (random rounding).
+ * The scales are those of halo_hadamard_quantize.  Everything else as there.
+ */
+halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                                        int axis, int blk, int qtype, const int8_t* signs,
+                                        const uint16_t* rand_bits, int64_t ld_rand, void* q_out,
+                                        int64_t ld_q, float* scales_out, void* stream);
+
+/*
  * Low-precision GEMM on codes with a dequantising epilogue:
  *     C[i, j] = (sum_k A[i, k] B[j, k]) * s_a[i] * s_b[j]
  * A is M x K and B is N x K (logically).  a_major / b_major give their

@@ -38,6 +38,38 @@ def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype):
     return int(exempt.sum()), int((diff & exempt).sum())
 
 
+def check_codes_stochastic(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, rand_bits, qtype, band=1e-4):
+    """Stochastic rounding: codes must match the oracle's except where the
+    decision is within `band` of flipping -- the random threshold u close to the
+    oracle's fraction p = (t - lo) / (hi - lo), or t close to a grid point (p
+    near 0 or 1) -- since the GPU forms t in fp32 (about 1e-7 relative).
+    Returns (#exempt, #exempt that differ)."""
+    g = u8(gpu_codes)
+    gs = gpu_scales.detach().cpu().numpy().astype(np.float64)
+    os_ = np.asarray(ora_scales, dtype=np.float64)
+    zero = os_ == 0
+    assert np.all(gs[zero] == 0)
+    rel = np.abs(gs[~zero] - os_[~zero]) / os_[~zero]
+    assert rel.size == 0 or rel.max() <= SCALE_REL
+    t = np.asarray(ora_t)
+    u = np.asarray(rand_bits, dtype=np.float64) / 65536.0
+    if qtype == oracle.INT8:
+        p = t - np.floor(t)
+    else:
+        a = np.abs(t)
+        quantum = np.where(a < 2.0**-6, 2.0**-9, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-300))) - 3))
+        p = (a - np.floor(a / quantum) * quantum) / quantum
+    exempt = (np.abs(u - p) < band) | (p < band) | (p > 1 - band)
+    diff = g != ora_codes
+    bad = diff & ~exempt
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        details = [(tuple(i), int(g[tuple(i)]), int(ora_codes[tuple(i)]), float(t[tuple(i)]), float(u[tuple(i)]))
+                   for i in idx]
+        raise AssertionError(f"{int(bad.sum())} stochastic code mismatches outside the band, e.g. {details}")
+    return int(exempt.sum()), int((diff & exempt).sum())
+
+
 def bf16_half_ulp(y: np.ndarray) -> np.ndarray:
     """Half the spacing of bf16 numbers (8 significant bits) at |y|."""
     a = np.abs(y)

@@ -126,3 +126,15 @@ def test_linear_host_validation(lib):
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 256, 0, FAKE, 0, FAKE, 0, FAKE, wsb, None) == BLOCK
     assert b(FAKE, FAKE, FAKE, 200, 256, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == SHAPE  # M % 128
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE
+
+
+def test_hadamard_quantize_ex_host_validation(lib):
+    f = lib.halo_hadamard_quantize_ex
+    # plain arguments are checked as for halo_hadamard_quantize
+    assert f(None, 256, 512, 512, 0, 128, 0, None, None, 0, FAKE, 512, FAKE, None) == NULL
+    assert f(FAKE, 256, 512, 512, 0, 64, 0, None, None, 0, FAKE, 512, FAKE, None) == BLOCK
+    # signs and random bits: alignment and stride
+    assert f(FAKE, 256, 512, 512, 0, 128, 0, MISALIGNED, None, 0, FAKE, 512, FAKE, None) == ALIGN
+    assert f(FAKE, 256, 512, 512, 0, 128, 0, None, MISALIGNED, 512, FAKE, 512, FAKE, None) == ALIGN
+    assert f(FAKE, 256, 512, 512, 0, 128, 0, None, FAKE, 500, FAKE, 512, FAKE, None) == SHAPE  # ld < cols
+    assert f(FAKE, 256, 512, 512, 0, 128, 0, None, FAKE, 516, FAKE, 512, FAKE, None) == ALIGN  # 1032-byte rows

@@ -275,3 +275,77 @@ def test_full_llama70b_layer_step_as_benchmarked(qtype):
         check_output(c[ri_t][:, cj_t], ref)
     del step
     torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------------- variants
+def _signs_t(n, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randint(0, 2, (n,), generator=g, dtype=torch.int8) * 2 - 1).to(torch.int8)
+
+
+def _rand_bits(rows, cols, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(0, 65536, (rows, cols), generator=g, dtype=torch.int32).to(torch.uint16)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("axis,rows,cols,blk", [(COLS, 300, 640, 128), (COLS, 64, 512, 256), (COLS, 7, 11008, 128),
+                                                (ROWS, 1024, 208, 128), (ROWS, 8320, 32, 128)])
+def test_random_sign_rotation_parity(qtype, axis, rows, cols, blk):
+    x = inputs.activations(rows, cols, seed=rows + cols + 5, device="cpu")
+    s = _signs_t(cols if axis == COLS else rows, seed=rows)
+    q, sc = halo.halo_hadamard_quantize_ex(_cuda(x), axis, blk, qtype, signs=_cuda(s))
+    torch.cuda.synchronize()
+    v = oracle.rotate_signed(x, blk, 1 if axis == COLS else 0, s.numpy())
+    codes, scales, t = oracle.quantize(v, axis=0 if axis == COLS else 1, qtype=qtype)
+    check_codes(q, sc, codes, scales, t, qtype)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("axis,rows,cols,blk", [(COLS, 300, 640, 128), (COLS, 64, 512, 256), (ROWS, 1024, 208, 128),
+                                                (ROWS, 8320, 32, 128)])
+def test_stochastic_rounding_parity(qtype, axis, rows, cols, blk):
+    x = inputs.activations(rows, cols, seed=rows * 3 + cols, device="cpu")
+    rb = _rand_bits(rows, cols, seed=cols)
+    q, sc = halo.halo_hadamard_quantize_ex(_cuda(x), axis, blk, qtype, rand_bits=_cuda(rb))
+    torch.cuda.synchronize()
+    v = oracle.rotate(x, blk, 1 if axis == COLS else 0)
+    codes, scales, t = oracle.quantize_stochastic(v, 0 if axis == COLS else 1, qtype, rb.numpy())
+    from tests._parity import check_codes_stochastic
+
+    n_ex, n_diff = check_codes_stochastic(q, sc, codes, scales, t, rb.numpy(), qtype)
+    assert n_ex < 0.01 * x.numel()
+
+
+def test_signs_and_stochastic_rounding_together_and_strided_random_bits():
+    rows, cols = 256, 1024
+    x = inputs.activations(rows, cols, seed=77, device="cpu")
+    s = _signs_t(cols, seed=78)
+    rb_full = _rand_bits(rows, cols + 64, seed=79)  # row stride cols + 64
+    rb = rb_full[:, :cols]
+    q, sc = halo.halo_hadamard_quantize_ex(_cuda(x), COLS, 128, INT8, signs=_cuda(s), rand_bits=_cuda(rb_full)[:, :cols])
+    torch.cuda.synchronize()
+    v = oracle.rotate_signed(x, 128, 1, s.numpy())
+    codes, scales, t = oracle.quantize_stochastic(v, 0, INT8, rb.contiguous().numpy())
+    from tests._parity import check_codes_stochastic
+
+    check_codes_stochastic(q, sc, codes, scales, t, rb.contiguous().numpy(), INT8)
+
+
+def test_random_sign_gemm_keeps_the_product():
+    """Both operands rotated with the same signs along K: the quantised GEMM
+    matches the oracle's signed-rotation GEMM, and stays close to X W^T."""
+    m, n, k = 384, 320, 640
+    x = inputs.activations(m, k, seed=81, device="cpu")
+    w = inputs.weights(n, k, seed=82, device="cpu")
+    s = _signs_t(k, seed=83)
+    qx, sx = halo.halo_hadamard_quantize_ex(_cuda(x), COLS, 128, INT8, signs=_cuda(s))
+    qw, sw = halo.halo_hadamard_quantize_ex(_cuda(w), COLS, 128, INT8, signs=_cuda(s))
+    y = halo.halo_qgemm(qx, sx, 0, qw, sw, 0, m, n, k, INT8, FP32)
+    torch.cuda.synchronize()
+    cx, osx, _ = oracle.quantize(oracle.rotate_signed(x, 128, 1, s.numpy()), 0, INT8)
+    cw, osw, _ = oracle.quantize(oracle.rotate_signed(w, 128, 1, s.numpy()), 0, INT8)
+    ref = oracle.dequant(oracle.gemm_i8(cx, cw).astype(np.float64), osx, osw)
+    check_output(y, ref)
+    exact = x.double().numpy() @ w.double().numpy().T
+    assert np.max(np.abs(ref - exact)) < 0.05 * np.max(np.abs(exact))
