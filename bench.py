@@ -518,6 +518,23 @@ def measure_rotq_shapes(repeats: int = 10):
     return {"measure": "rotate+quantise per shape", "block": BLK, "results": out}
 
 
+# ------------------------------------------------------------------ multi-rank
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Device-timed region of this rank -> the maximum over all ranks (the
+    job's time).  One all-reduce; every rank calls it in the same place."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ops_per_step: int, steps: int, world: int, ms_total: float) -> float:
+    """Whole-job throughput in TOPS: every rank runs `steps` steps of the same
+    work (replicas, weak scaling), over the max-over-ranks time."""
+    return ops_per_step * steps * world / (ms_total * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------------- main
 WORKLOADS = {
     "llama70b_layer_fwd_bwd": (inputs.LLAMA70B_LAYER, ("fwd", "dx", "dw")),
@@ -613,11 +630,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(end)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
     st, site = halo.halo_device_error()
     if st != halo.HALO_OK:
         raise RuntimeError(f"device error in the timed region at site {site:#x}")
@@ -635,7 +648,7 @@ def main():
 
     ops_step = step.ops_per_step()
     ms_step = ms_total / args.steps
-    value = ops_step * args.steps * world / (ms_total * 1e-3) / 1e12
+    value = job_throughput(ops_step, args.steps, world, ms_total)
     gemm_tops = step.gemm_ops() * args.steps / (gemm_ms * 1e-3) / 1e12
     rotq_gbs = step.rotq_bytes() * args.steps / (rotq_ms * 1e-3) / 1e9
     pk = peaks()

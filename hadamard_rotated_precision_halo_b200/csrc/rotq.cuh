@@ -327,9 +327,41 @@ __global__ void __launch_bounds__(256)
     if (chunk == 0) p.scales[row] = row_amax * p.scale_mult;
     if (is_active) {
       uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
-      const uint4* rnd = EXT ? reinterpret_cast<const uint4*>(p.ex.rand + row * p.ex.ld_rand +
-                                                                static_cast<int64_t>(chunk) * 128)
-                             : nullptr;
+      if (EXT && p.ex.rand != nullptr) {
+        // Stochastic rounding: the chunk's 128 random values in two batches of
+        // 8 vectors, loaded before the code stores so that the loads overlap.
+        const uint4* rnd =
+            reinterpret_cast<const uint4*>(p.ex.rand + row * p.ex.ld_rand + static_cast<int64_t>(chunk) * 128);
+#pragma unroll
+        for (int kb = 0; kb < 8; kb += 4) {
+          uint4 rv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) rv[i] = __ldg(rnd + 2 * kb + i);
+#pragma unroll
+          for (int k = kb; k < kb + 4; ++k) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              // elements 16k + 4j .. +3: random halves 4(j%2) .. +3 of vector 2k + j/2
+              const float2 a = v[8 * k + 2 * j];
+              const float2 b = v[8 * k + 2 * j + 1];
+              const uint4 rq = rv[2 * (k - kb) + j / 2];
+              const uint32_t r01 = (j & 1) ? rq.z : rq.x;
+              const uint32_t r23 = (j & 1) ? rq.w : rq.y;
+              const float u0 = rand_unit(r01 & 0xFFFFu), u1 = rand_unit(r01 >> 16);
+              const float u2 = rand_unit(r23 & 0xFFFFu), u3 = rand_unit(r23 >> 16);
+              if (QT == 0) {
+                w[j] = pack4_int8(q_int8_sr(a.x * r, u0), q_int8_sr(a.y * r, u1), q_int8_sr(b.x * r, u2),
+                                  q_int8_sr(b.y * r, u3));
+              } else {
+                w[j] = e4m3x2_bits(e4m3_sr_value(a.x * r, u0), e4m3_sr_value(a.y * r, u1)) |
+                       (e4m3x2_bits(e4m3_sr_value(b.x * r, u2), e4m3_sr_value(b.y * r, u3)) << 16);
+              }
+            }
+            dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         uint32_t w[4];
@@ -337,22 +369,6 @@ __global__ void __launch_bounds__(256)
         for (int j = 0; j < 4; ++j) {
           const float2 a = v[8 * k + 2 * j];
           const float2 b = v[8 * k + 2 * j + 1];
-          if (EXT && p.ex.rand != nullptr) {
-            // elements 16k + 4j .. +3: random halves 4(j%2) .. +3 of vector 2k + j/2
-            const uint4 rv = __ldg(rnd + 2 * k + j / 2);
-            const uint32_t r01 = (j & 1) ? rv.z : rv.x;
-            const uint32_t r23 = (j & 1) ? rv.w : rv.y;
-            const float u0 = rand_unit(r01 & 0xFFFFu), u1 = rand_unit(r01 >> 16);
-            const float u2 = rand_unit(r23 & 0xFFFFu), u3 = rand_unit(r23 >> 16);
-            if (QT == 0) {
-              w[j] = pack4_int8(q_int8_sr(a.x * r, u0), q_int8_sr(a.y * r, u1), q_int8_sr(b.x * r, u2),
-                                q_int8_sr(b.y * r, u3));
-            } else {
-              w[j] = e4m3x2_bits(e4m3_sr_value(a.x * r, u0), e4m3_sr_value(a.y * r, u1)) |
-                     (e4m3x2_bits(e4m3_sr_value(b.x * r, u2), e4m3_sr_value(b.y * r, u3)) << 16);
-            }
-            continue;
-          }
           if (QT == 0) {
             w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r),
                               q_int8_bits(b.y, r));
@@ -361,6 +377,7 @@ __global__ void __launch_bounds__(256)
           }
         }
         dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
       }
     }
     fence_proxy_async_smem();
@@ -424,19 +441,32 @@ template <int QT, int EXT = 0>
 __device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
                                                  int h, const uint16_t* rnd = nullptr, int64_t ld_rand = 0) {
   uint16_t* outw = reinterpret_cast<uint16_t*>(tile);
+  if (EXT && rnd != nullptr) {
+    // Random bits in batches of 16 rows, loaded before the code stores so that
+    // the loads overlap instead of waiting one by one behind each store.
+#pragma unroll
+    for (int i0 = 0; i0 < 64; i0 += 16) {
+      uint32_t rb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        rb[i] = __ldg(reinterpret_cast<const uint32_t*>(rnd + (2 * (i0 + i) + h) * ld_rand));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float u0 = rand_unit(rb[i] & 0xFFFFu), u1 = rand_unit(rb[i] >> 16);
+        const float2 x = v[i0 + i];
+        uint32_t code;
+        if (QT == 0)
+          code = __byte_perm(q_int8_sr(x.x * r0, u0), q_int8_sr(x.y * r1, u1), 0x0040) & 0xFFFFu;
+        else
+          code = e4m3x2_bits(e4m3_sr_value(x.x * r0, u0), e4m3_sr_value(x.y * r1, u1));
+        outw[(2 * (i0 + i) + h) * 16 + pcol] = static_cast<uint16_t>(code);
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     uint32_t code;
-    if (EXT && rnd != nullptr) {
-      const uint32_t rb = __ldg(reinterpret_cast<const uint32_t*>(rnd + (2 * i + h) * ld_rand));
-      const float u0 = rand_unit(rb & 0xFFFFu), u1 = rand_unit(rb >> 16);
-      if (QT == 0)
-        code = __byte_perm(q_int8_sr(v[i].x * r0, u0), q_int8_sr(v[i].y * r1, u1), 0x0040) & 0xFFFFu;
-      else
-        code = e4m3x2_bits(e4m3_sr_value(v[i].x * r0, u0), e4m3_sr_value(v[i].y * r1, u1));
-      outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
-      continue;
-    }
     if (QT == 0) {
       code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
     } else {
