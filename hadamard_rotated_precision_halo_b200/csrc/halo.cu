@@ -295,8 +295,7 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
   Cols1Kernel kern = cols_1pass_kernel(qtype, nw, ext);
 
   // Persistent: as many clusters as fit at once (each loops over strips).
-  Launch L(dim3(cl, 1, 1), dim3(32 * nw), static_cast<size_t>(nw) * (2 * kColsInBytes + kColsOutBytes) + 128,
-           stream, cl);
+  Launch L(dim3(cl, 1, 1), dim3(32 * nw), static_cast<size_t>(nw) * (2 * kColsInBytes) + 128, stream, cl);
   int max_clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &L.cfg) != cudaSuccess || max_clusters < 1) {
     (void)cudaGetLastError();
@@ -348,7 +347,7 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
   p.ex = ex;
-  const size_t smem = static_cast<size_t>(warps) * (kColsStages * kColsInBytes + 2 * kColsOutBytes) + 128;
+  const size_t smem = static_cast<size_t>(warps) * (kColsStages * kColsInBytes) + 128;
 
   Launch L(dim3(cl, strips, 1), dim3(32 * warps), smem, stream, cl);
   HALO_CUDA(cudaLaunchKernelEx(&L.cfg, cols_2pass_kernel(qtype, ext), tm_x, tm_q, p));

@@ -468,7 +468,9 @@ __device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v
   for (int i = 0; i < 64; ++i) {
     uint32_t code;
     if (QT == 0) {
-      code = __byte_perm(q_int8_bits(v[i].x, r0), q_int8_bits(v[i].y, r1), 0x0040) & 0xFFFFu;
+      // Both columns in one packed FMA (same rounding as q_int8_bits).
+      const float2 t = __ffma2_rn(v[i], make_float2(r0, r1), make_float2(12582912.0f, 12582912.0f));
+      code = __byte_perm(__float_as_uint(t.x), __float_as_uint(t.y), 0x0040);  // low 16 bits stored
     } else {
       code = e4m3x2_bits(v[i].x * r0, v[i].y * r1);
     }
@@ -487,7 +489,7 @@ struct RotqColsParams {
 };
 
 template <int QT, int EXT>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, EXT ? 2 : 3)
     rotq_cols_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                      RotqColsParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -505,7 +507,6 @@ __global__ void __launch_bounds__(128)
   const int c0 = blockIdx.y * kColsStrip;
 
   uint8_t* s_in = smem + warp * (kColsStages * kColsInBytes);
-  uint8_t* s_out = smem + p.warps * (kColsStages * kColsInBytes) + warp * (2 * kColsOutBytes);
 
   if (threadIdx.x < kColsStrip) s_part[threadIdx.x] = 0u;
   if (lane == 0) {
@@ -587,10 +588,14 @@ __global__ void __launch_bounds__(128)
     r1 = cm1 > 0.f ? __fdiv_rn(p.qmax, cm1) : 0.f;
   }
 
+  // Pass 2.  The codes of a block go into the input stage it was read from;
+  // the other stage held the previous block, whose codes were stored from it
+  // at the end of the previous iteration: once that store has read them, the
+  // stage is refilled with the next block.  (The first two pass-2 blocks were
+  // requested during pass 1.)
   for (int j = nmine; j < nseq && !failed; ++j) {
     const int s = j % kColsStages;
     const uint32_t ph = (j / kColsStages) & 1u;
-    const int ob = (j - nmine) & 1;
     const bool ok = mbar_wait(&bars[warp][s], ph, kSiteRotqColsLoad);
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
@@ -598,23 +603,23 @@ __global__ void __launch_bounds__(128)
     const int bq = first + step * (j - nmine);
     cols_load_fwht<EXT>(blkw, pcol, h, v, EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(bq) * 128 : nullptr);
     __syncwarp();
-    if (lane == 0) {
-      if (j + kColsStages < nseq) issue(j + kColsStages);
-      bulk_wait_read<1>();  // code buffer `ob` (used two blocks ago) is free again
-    }
     cols_fwht_rest(v);
-    __syncwarp();
+    if (lane == 0 && j > nmine && j + 1 < nseq) {
+      bulk_wait_read<0>();
+      issue(j + 1);
+    }
+    uint8_t* s_codes = s_in + s * kColsInBytes;  // every lane has read this stage (warp sync above)
     {
       const bool col_ok = c0 + 2 * pcol < p.cols;
       const uint16_t* rnd = EXT && p.ex.rand && col_ok
                                 ? p.ex.rand + static_cast<int64_t>(bq) * 128 * p.ex.ld_rand + c0 + 2 * pcol
                                 : nullptr;
-      cols_write_codes<QT, EXT>(s_out + ob * kColsOutBytes, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
+      cols_write_codes<QT, EXT>(s_codes, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
     }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(&tm_q, s_out + ob * kColsOutBytes, c0, bq * 128);
+      tma_store_2d(&tm_q, s_codes, c0, bq * 128);
       bulk_commit();
     }
   }
@@ -628,7 +633,10 @@ __global__ void __launch_bounds__(128)
 // 128-row blocks split over a cluster of at most 16 CTAs of NW <= 4 warps, one
 // block per warp (R = CL * NW * 128 <= 8192 rows).  Every rotated value stays
 // in registers while the column maxima are reduced, so the input is read once
-// and the codes written once.
+// and the codes written once.  The codes of a strip go into the input stage
+// that strip was read from (the store has read them before the stage is
+// refilled), so a warp holds 16 KB of shared memory and three 4-warp CTAs fit
+// on an SM.
 //
 // Column-max reduction per strip: warps -> CTA with shared-memory atomics and
 // one CTA barrier; then the CTA's 32 partial maxima (128 bytes) go to every
@@ -638,7 +646,7 @@ __global__ void __launch_bounds__(128)
 // fence in the loop.  Two slot buffers alternate over strips: a peer writes
 // strip k+2 only after every CTA has sent strip k+1, which each CTA does only
 // after it has read strip k.  The cluster is persistent over strips; each warp
-// prefetches its block of the next two strips with TMA.
+// keeps its block of the next strip in flight with TMA.
 // ------------------------------------------------------------------------------------------
 struct RotqCols1Params {
   float* scales;
@@ -652,7 +660,7 @@ struct RotqCols1Params {
 enum : unsigned int { kSiteRotqCols1Load = 0x202, kSiteRotqCols1Reduce = 0x203 };
 
 template <int QT, int NW, int EXT>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
     rotq_cols_1pass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
                            RotqCols1Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -672,7 +680,6 @@ __global__ void __launch_bounds__(NW * 32)
   const uint32_t slot_bytes = csize * kColsStrip * 4;
 
   uint8_t* s_in = smem + warp * (2 * kColsInBytes);
-  uint8_t* s_out = smem + NW * (2 * kColsInBytes) + warp * kColsOutBytes;
 
   if (threadIdx.x < 2 * kColsStrip) (&s_red[0][0])[threadIdx.x] = 0u;
   if (lane == 0) {
@@ -725,8 +732,13 @@ __global__ void __launch_bounds__(NW * 32)
       for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
     }
     __syncwarp();
-    if (lane == 0 && !dead && k + 2 < nmine) issue(k + 2);
     cols_fwht_rest(v);
+    // The other stage held strip k - 1, whose codes were stored from it at the
+    // end of the previous iteration: once that store has read them, refill it.
+    if (lane == 0 && !dead && k >= 1 && k + 1 < nmine) {
+      bulk_wait_read<0>();
+      issue(k + 1);
+    }
     const float2 mm = absmax64_cols(v);
     float m0 = mm.x, m1 = mm.y;
     m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
@@ -761,19 +773,18 @@ __global__ void __launch_bounds__(NW * 32)
       if (c0 + 2 * pcol < p.cols) p.scales[c0 + 2 * pcol] = cm0 * p.scale_mult;
       if (c0 + 2 * pcol + 1 < p.cols) p.scales[c0 + 2 * pcol + 1] = cm1 * p.scale_mult;
     }
-    if (lane == 0) bulk_wait_read<0>();  // the previous strip's store has read the code tile
-    __syncwarp();
+    uint8_t* s_codes = s_in + par * kColsInBytes;  // every lane has read this stage (warp sync above)
     {
       const bool col_ok = c0 + 2 * pcol < p.cols;
       const uint16_t* rnd = EXT && p.ex.rand && col_ok
                                 ? p.ex.rand + static_cast<int64_t>(blk) * 128 * p.ex.ld_rand + c0 + 2 * pcol
                                 : nullptr;
-      cols_write_codes<QT, EXT>(s_out, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
+      cols_write_codes<QT, EXT>(s_codes, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
     }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(&tm_q, s_out, c0, blk * 128);
+      tma_store_2d(&tm_q, s_codes, c0, blk * 128);
       bulk_commit();
     }
   }

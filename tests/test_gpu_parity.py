@@ -349,3 +349,42 @@ def test_random_sign_gemm_keeps_the_product():
     check_output(y, ref)
     exact = x.double().numpy() @ w.double().numpy().T
     assert np.max(np.abs(ref - exact)) < 0.05 * np.max(np.abs(exact))
+
+
+# ------------------------------------------------------------------- edge cases
+def test_single_token_forward_and_tiny_backward():
+    x = inputs.activations(1, 256, seed=91, device="cpu")
+    w = inputs.weights(16, 256, seed=92, device="cpu")
+    y = halo.halo_linear_fwd(_cuda(x), _cuda(w), 128, INT8, FP32)
+    torch.cuda.synchronize()
+    check_output(y, oracle.linear_fwd(x, w, 128, INT8))
+    m, n, k = 128, 128, 16  # one 128-block along tokens and along N
+    dy = inputs.grads(m, n, seed=93, device="cpu")
+    xb = inputs.activations(m, k, seed=94, device="cpu")
+    wb = inputs.weights(n, k, seed=95, device="cpu")
+    dx, dw = halo.halo_linear_bwd(_cuda(dy), _cuda(xb), _cuda(wb), 128, INT8, FP32, FP32)
+    torch.cuda.synchronize()
+    check_output(dx, oracle.linear_bwd_dx(dy, wb, 128, INT8))
+    check_output(dw, oracle.linear_bwd_dw(dy, xb, 128, INT8))
+
+
+def test_all_zero_operands_give_zero_scales_codes_and_outputs():
+    x = torch.zeros((256, 512), dtype=torch.bfloat16, device="cuda")
+    w = inputs.weights(128, 512, seed=96, device="cuda")
+    for axis in (COLS, ROWS):
+        q, s = halo.halo_hadamard_quantize(x, axis, 128, INT8)
+        torch.cuda.synchronize()
+        assert torch.all(s == 0) and torch.all(q.view(torch.uint8) == 0)
+    y = halo.halo_linear_fwd(x, w, 128, INT8, FP32)
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+def test_rotq_rows_longest_row(qtype):
+    """32768 elements per row: 256 chunks, a row group of 8 warps (the largest)."""
+    x = inputs.activations(6, 32768, seed=97, device="cpu")
+    q, s = halo.halo_hadamard_quantize(_cuda(x), COLS, 128, qtype)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle_operand(x, 1, 128, qtype)
+    check_codes(q, s, codes, scales, t, qtype)
