@@ -534,6 +534,26 @@ def measure_rotq_shapes(repeats: int = 10):
                 out.append({"direction": name, "shape": [r, c], "qtype": "int8" if qt == 0 else "e4m3",
                             "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
             del x, q, sc
+    # Both encodings from one read (halo_hadamard_quantize_dual): 2 B in + 1 B
+    # per code set per element, 4 B per scale of each set.
+    for r, c in ROTQ_SHAPES["along_contiguous_dim"]:
+        x = inputs.activations(r, c, seed=1, device="cuda")
+        outs = halo.halo_hadamard_quantize_dual(x, BLK)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(repeats):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            halo.halo_hadamard_quantize_dual(x, BLK, *outs)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = sorted(ts)[len(ts) // 2]
+        nbytes = 4 * x.numel() + 8 * r
+        out.append({"direction": "along_contiguous_dim", "shape": [r, c], "qtype": "int8+e4m3 (one read)",
+                    "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
+        del x, outs
     # The variants (halo_hadamard_quantize_ex): random signs along the rotated
     # dimension and stochastic rounding from 16 random bits per element (which
     # add 2 B per element of input traffic).

@@ -40,6 +40,7 @@ HALO_MAJOR_MN = 1
 EXPORTS = (
     "halo_hadamard_quantize",
     "halo_hadamard_quantize_ex",
+    "halo_hadamard_quantize_dual",
     "halo_qgemm",
     "halo_workspace_size",
     "halo_linear_fwd",
@@ -79,6 +80,8 @@ def lib():
     L.halo_hadamard_quantize.restype = I
     L.halo_hadamard_quantize_ex.argtypes = [P, I64, I64, I64, I, I, I, P, P, I64, P, I64, P, P]
     L.halo_hadamard_quantize_ex.restype = I
+    L.halo_hadamard_quantize_dual.argtypes = [P, I64, I64, I64, I, P, I64, P, P, I64, P, P]
+    L.halo_hadamard_quantize_dual.restype = I
     L.halo_qgemm.argtypes = [P, P, I, I64, P, P, I, I64, I64, I64, I64, I, P, I, I64, P]
     L.halo_qgemm.restype = I
     L.halo_workspace_size.argtypes = [I64, I64, I64, I]
@@ -162,6 +165,26 @@ def halo_hadamard_quantize_ex(x: torch.Tensor, axis: int, blk: int, qtype: int, 
                                          _stream(stream))
     _check(st, "halo_hadamard_quantize_ex")
     return q_out, scales_out
+
+
+def halo_hadamard_quantize_dual(x: torch.Tensor, blk: int, q_int8=None, scales_int8=None, q_e4m3=None,
+                                scales_e4m3=None, stream=None):
+    """Rotate along the contiguous dim once, quantise to INT8 and to E4M3;
+    returns (int8 codes, int8 scales, e4m3 codes, e4m3 scales)."""
+    rows, cols = x.shape
+    if q_int8 is None:
+        q_int8 = torch.empty((rows, cols), dtype=_code_dtype(HALO_Q_INT8), device=x.device)
+    if q_e4m3 is None:
+        q_e4m3 = torch.empty((rows, cols), dtype=_code_dtype(HALO_Q_E4M3), device=x.device)
+    if scales_int8 is None:
+        scales_int8 = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if scales_e4m3 is None:
+        scales_e4m3 = torch.empty(rows, dtype=torch.float32, device=x.device)
+    st = lib().halo_hadamard_quantize_dual(_ptr(x), rows, cols, x.stride(0), blk, _ptr(q_int8), q_int8.stride(0),
+                                           _ptr(scales_int8), _ptr(q_e4m3), q_e4m3.stride(0), _ptr(scales_e4m3),
+                                           _stream(stream))
+    _check(st, "halo_hadamard_quantize_dual")
+    return q_int8, scales_int8, q_e4m3, scales_e4m3
 
 
 def halo_qgemm(a_q, s_a, a_major, b_q, s_b, b_major, m, n, k, qtype, otype, c=None, stream=None):

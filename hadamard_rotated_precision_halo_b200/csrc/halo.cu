@@ -65,13 +65,15 @@ cudaError_t set_smem_attr(K kernel, int optin) {
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
-typedef void (*RowsKernel)(const CUtensorMap, const CUtensorMap, RotqRowsParams);
+typedef void (*RowsKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, RotqRowsParams);
 typedef void (*Cols1Kernel)(const CUtensorMap, const CUtensorMap, RotqCols1Params);
 typedef void (*Cols2Kernel)(const CUtensorMap, const CUtensorMap, RotqColsParams);
 
 // `ext`: the instantiation that reads the variants' optional inputs (signs,
 // random bits); the plain path is compiled without them.
+// qtype kQtDual (2): INT8 and E4M3 codes from one read (plain path only).
 RowsKernel rows_kernel(int blk, int qtype, bool ext) {
+  if (qtype == kQtDual) return blk == 128 ? rotq_rows_kernel<128, kQtDual, 0> : rotq_rows_kernel<256, kQtDual, 0>;
   if (blk == 128) {
     if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<128, 0, 1> : rotq_rows_kernel<128, 0, 0>;
     return ext ? rotq_rows_kernel<128, 1, 1> : rotq_rows_kernel<128, 1, 0>;
@@ -129,6 +131,8 @@ halo_status_t device_setup(int* dev_out) {
     }
     int optin = 0;
     HALO_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    HALO_CUDA(set_smem_attr(rows_kernel(128, kQtDual, false), optin));
+    HALO_CUDA(set_smem_attr(rows_kernel(256, kQtDual, false), optin));
     for (int e = 0; e < 2; ++e) {
       for (int qt = 0; qt < 2; ++qt) {
         HALO_CUDA(set_smem_attr(rows_kernel(128, qt, e), optin));
@@ -212,9 +216,13 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
 }
 
 // ------------------------------------------------------------------------ rotq launches
+// qtype kQtDual: q / ld_q / scales take the INT8 output, q2 / ld_q2 / scales2
+// the E4M3 one (unused otherwise).
 halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
                                void* q, int64_t ld_q, float* scales, const RotqExtras& ex, bool ext,
-                               cudaStream_t stream, int dev) {
+                               cudaStream_t stream, int dev, void* q2 = nullptr, int64_t ld_q2 = 0,
+                               float* scales2 = nullptr) {
+  const bool dual = qtype == kQtDual;
   const int nb = static_cast<int>(cols / 128);
   // A row group of ceil(nb / 32) warps owns one row at a time; 4 warps per
   // CTA when a group fits in 4, else one group per CTA (up to 8 warps).
@@ -222,7 +230,7 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   const int groups = gw <= 4 ? 4 / gw : 1;
   const int threads = groups * gw * 32;
 
-  CUtensorMap tm_x, tm_q;
+  CUtensorMap tm_x, tm_q, tm_q2;
   {
     cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
@@ -238,8 +246,14 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
     halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != HALO_OK) return st;
+    tm_q2 = tm_q;
+    if (dual) {
+      strides[1] = static_cast<cuuint64_t>(ld_q2);
+      st = encode(&tm_q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != HALO_OK) return st;
+    }
   }
-  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw) + 128;  // + alignment slack
+  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw, dual ? 2 : 1) + 128;  // + alignment slack
 
   RotqRowsParams p;
   p.scales = scales;
@@ -247,9 +261,11 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   p.nb = nb;
   p.gw = gw;
   p.groups = groups;
-  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.qmax = qtype == HALO_Q_E4M3 ? 448.f : 127.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(static_cast<double>(blk))));
   p.ex = ex;
+  p.scales2 = scales2;
+  p.scale_mult2 = static_cast<float>(1.0 / (448.0 * sqrt(static_cast<double>(blk))));
 
   RowsKernel kern = rows_kernel(blk, qtype, ext);
   int per_sm = 0;
@@ -258,7 +274,7 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   const int64_t ctas_needed = (rows + groups - 1) / groups;
   const int grid = static_cast<int>(std::min<int64_t>(ctas_needed, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
   Launch L(dim3(grid), dim3(threads), smem, stream, 0);
-  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, tm_q2, p));
   return HALO_OK;
 }
 
@@ -591,6 +607,26 @@ halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t c
                                      void* stream) {
   return halo_hadamard_quantize_ex(x_bf16, rows, cols, ld_x, axis, blk, qtype, nullptr, nullptr, 0, q_out, ld_q,
                                    scales_out, stream);
+}
+
+halo_status_t halo_hadamard_quantize_dual(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
+                                          void* q_int8, int64_t ld_q8, float* scales_int8, void* q_e4m3,
+                                          int64_t ld_qf8, float* scales_e4m3, void* stream) {
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_COLS, blk, HALO_Q_INT8, q_int8,
+                                             ld_q8, scales_int8);
+  if (st != HALO_OK) return st;
+  st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_COLS, blk, HALO_Q_E4M3, q_e4m3, ld_qf8,
+                               scales_e4m3);
+  if (st != HALO_OK) return st;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  RotqExtras ex;
+  ex.signs = nullptr;
+  ex.rand = nullptr;
+  ex.ld_rand = 0;
+  return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, kQtDual, q_int8, ld_q8, scales_int8, ex, false,
+                          static_cast<cudaStream_t>(stream), dev, q_e4m3, ld_qf8, scales_e4m3);
 }
 
 halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,

@@ -199,12 +199,21 @@ struct RotqRowsParams {
   float qmax;
   float scale_mult;  // 1 / (qmax * sqrt(blk))
   RotqExtras ex;     // EXT = 1 only
+  float* scales2;    // QT = 2 only: the E4M3 scales (`scales` holds the INT8 ones)
+  float scale_mult2; // QT = 2 only: 1 / (448 * sqrt(blk))
 };
 
-// Shared-memory bytes of one row group: 2 input stages and one code tile.
+// QT = 2: both code sets from one read of the input -- INT8 codes with their
+// scales through tm_q / scales, E4M3 codes with theirs through tm_q2 / scales2.
+constexpr int kQtDual = 2;
+
+// Shared-memory bytes of one row group: 2 input stages and one code tile (two
+// for the dual output).
 __host__ __device__ inline uint32_t rows_group_in_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsInSlot; }
 __host__ __device__ inline uint32_t rows_group_out_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsOutSlot; }
-__host__ __device__ inline uint32_t rows_group_smem(int gw) { return 2 * rows_group_in_bytes(gw) + rows_group_out_bytes(gw); }
+__host__ __device__ inline uint32_t rows_group_smem(int gw, int ntiles = 1) {
+  return 2 * rows_group_in_bytes(gw) + ntiles * rows_group_out_bytes(gw);
+}
 
 __device__ __forceinline__ void group_sync(int gw, int grp) {
   if (gw == 1)
@@ -216,7 +225,8 @@ __device__ __forceinline__ void group_sync(int gw, int grp) {
 template <int BLK, int QT, int EXT>
 __global__ void __launch_bounds__(256)
     rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
-                     RotqRowsParams p) {
+                     const __grid_constant__ CUtensorMap tm_q2, RotqRowsParams p) {
+  constexpr int kTiles = QT == kQtDual ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   __shared__ uint64_t full_bar[8][2];
@@ -231,8 +241,9 @@ __global__ void __launch_bounds__(256)
   const bool is_active = chunk < p.nb;
   const bool leader = (wig == 0 && lane == 0);
   const uint32_t in_bytes = static_cast<uint32_t>(p.nb) * kRowsInSlot;  // one row's box
-  uint8_t* g_in = smem + grp * rows_group_smem(gw);
+  uint8_t* g_in = smem + grp * rows_group_smem(gw, kTiles);
   uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw);
+  uint8_t* g_out2 = g_out + rows_group_out_bytes(gw);  // QT = 2 only
 
   if (leader) {
     mbar_init(&full_bar[grp][0], 1);
@@ -240,6 +251,7 @@ __global__ void __launch_bounds__(256)
     fence_mbar_init();
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_q);
+    if (QT == kQtDual) prefetch_tmap(&tm_q2);
   }
   __syncthreads();
   griddep_wait();  // inputs written and codes read by the previous kernel
@@ -325,7 +337,27 @@ __global__ void __launch_bounds__(256)
     const float row_amax = __uint_as_float(wmax);
     const float r = row_amax > 0.f ? __fdiv_rn(p.qmax, row_amax) : 0.f;
     if (chunk == 0) p.scales[row] = row_amax * p.scale_mult;
-    if (is_active) {
+    if (QT == kQtDual) {
+      const float r2 = row_amax > 0.f ? __fdiv_rn(448.0f, row_amax) : 0.f;
+      if (chunk == 0) p.scales2[row] = row_amax * p.scale_mult2;
+      if (is_active) {
+        uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
+        uint4* dst2 = reinterpret_cast<uint4*>(g_out2 + chunk * kRowsOutSlot);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint32_t w[4], w2[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = v[8 * k + 2 * j];
+            const float2 b = v[8 * k + 2 * j + 1];
+            w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r), q_int8_bits(b.y, r));
+            w2[j] = e4m3x2_bits(a.x * r2, a.y * r2) | (e4m3x2_bits(b.x * r2, b.y * r2) << 16);
+          }
+          dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst2[k] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+        }
+      }
+    } else if (is_active) {
       uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
       if (EXT && p.ex.rand != nullptr) {
         // Stochastic rounding: the chunk's 128 random values in two batches of
@@ -384,7 +416,8 @@ __global__ void __launch_bounds__(256)
     group_sync(gw, grp);
     if (leader) {
       tma_store_3d(&tm_q, g_out, 0, 0, static_cast<int32_t>(row));
-      bulk_commit();
+      if (QT == kQtDual) tma_store_3d(&tm_q2, g_out2, 0, 0, static_cast<int32_t>(row));
+      bulk_commit();  // one group for both stores: the wait above covers both tiles
     }
   }
   if (leader) bulk_wait<0>();

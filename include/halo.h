@@ -124,6 +124,23 @@ halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_
                                         int64_t ld_q, float* scales_out, void* stream);
 
 /*
+ * Both 8-bit encodings of one rotation from a single read of X: the block
+ * rotation along the contiguous dimension (HALO_AXIS_COLS) of
+ * halo_hadamard_quantize, quantised per row to INT8 (codes q_int8 [rows, cols],
+ * row stride ld_q8 bytes, scales_int8 [rows] = amax / (127 sqrt(blk))) and to
+ * E4M3 (q_e4m3, ld_qf8, scales_e4m3 [rows] = amax / (448 sqrt(blk))).  Each
+ * output equals what halo_hadamard_quantize writes for its qtype, byte for
+ * byte; the input is read once instead of twice.  The two outputs must not
+ * overlap.  Arguments, alignment rules and errors as for
+ * halo_hadamard_quantize (axis HALO_AXIS_COLS, blk 128 or 256).
+ * Defined by: HALO paper page ("key design": INT8 or FP8 for every matmul);
+ * QWHA page sec. 2.1-2.2 (Walsh-Hadamard transform, symmetric quantiser).
+ */
+halo_status_t halo_hadamard_quantize_dual(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                                          int blk, void* q_int8, int64_t ld_q8, float* scales_int8,
+                                          void* q_e4m3, int64_t ld_qf8, float* scales_e4m3, void* stream);
+
+/*
  * Low-precision GEMM on codes with a dequantising epilogue:
  *     C[i, j] = (sum_k A[i, k] B[j, k]) * s_a[i] * s_b[j]
  * A is M x K and B is N x K (logically).  a_major / b_major give their

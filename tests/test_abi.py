@@ -138,3 +138,20 @@ def test_hadamard_quantize_ex_host_validation(lib):
     assert f(FAKE, 256, 512, 512, 0, 128, 0, None, MISALIGNED, 512, FAKE, 512, FAKE, None) == ALIGN
     assert f(FAKE, 256, 512, 512, 0, 128, 0, None, FAKE, 500, FAKE, 512, FAKE, None) == SHAPE  # ld < cols
     assert f(FAKE, 256, 512, 512, 0, 128, 0, None, FAKE, 516, FAKE, 512, FAKE, None) == ALIGN  # 1032-byte rows
+
+
+def test_hadamard_quantize_dual_host_validation(lib):
+    f = lib.halo_hadamard_quantize_dual
+    ok = (FAKE, 256, 512, 512, 128, FAKE, 512, FAKE, FAKE, 512, FAKE, None)
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a0=None) == NULL
+    assert call(a5=None) == NULL        # INT8 codes
+    assert call(a10=None) == NULL       # E4M3 scales
+    assert call(a4=64) == BLOCK
+    assert call(a2=500, a3=512) == SHAPE
+    assert call(a8=MISALIGNED) == ALIGN
+    assert call(a9=520) == ALIGN        # E4M3 row stride not a multiple of 16

@@ -351,6 +351,36 @@ def test_random_sign_gemm_keeps_the_product():
     assert np.max(np.abs(ref - exact)) < 0.05 * np.max(np.abs(exact))
 
 
+# ------------------------------------------------------------- dual INT8 + E4M3 output
+@pytest.mark.parametrize("rows,cols,blk", [(300, 640, 128), (130, 512, 256), (3, 28672, 128)])
+def test_rotq_dual_parity(rows, cols, blk):
+    x = inputs.activations(rows, cols, seed=rows + cols, device="cpu")
+    x[min(2, rows - 1)] = 0
+    xd = _cuda(x)
+    q8, s8, qf, sf = halo.halo_hadamard_quantize_dual(xd, blk)
+    torch.cuda.synchronize()
+    for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
+        codes, scales, t = oracle_operand(x, 1, blk, qt)
+        check_codes(q, s, codes, scales, t, qt)
+        # byte for byte what the single-output call writes
+        q1, s1 = halo.halo_hadamard_quantize(xd, COLS, blk, qt)
+        torch.cuda.synchronize()
+        assert torch.equal(q1.view(torch.uint8), q.view(torch.uint8)) and torch.equal(s1, s)
+
+
+def test_rotq_dual_full_size_16384x4096():
+    """The standalone rotate+quantise workload, both encodings from one read,
+    checked on sampled rows (each row depends on that row alone)."""
+    x = inputs.activations(16384, 4096, seed=2, device="cuda")
+    q8, s8, qf, sf = halo.halo_hadamard_quantize_dual(x, 128)
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(_sample(16384, 256, 5)).cuda()
+    xs = x[rows].cpu()
+    for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
+        codes, scales, t = oracle_operand(xs, 1, 128, qt)
+        check_codes(q[rows], s[rows], codes, scales, t, qt)
+
+
 # ------------------------------------------------------------------- edge cases
 def test_single_token_forward_and_tiny_backward():
     x = inputs.activations(1, 256, seed=91, device="cpu")
