@@ -121,14 +121,39 @@ def fwht(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def padded_length(n: int, blk: int) -> int:
+    """Length of a dimension of n elements after zero-padding to whole blocks."""
+    return -(-n // blk) * blk
+
+
+def pad_to_blocks(x, blk: int, axis: int) -> np.ndarray:
+    """Zero-pad a bf16 matrix along its rotated dimension to a multiple of blk
+    (QWHA page sec. 3.1 and 5: inputs whose length is not the transform's are
+    filled up with zeros before the transform; with block-local rotations only
+    the last block is filled).  axis=1: pad the columns; axis=0: pad the rows.
+    bf16 bit patterns in, bf16 bit patterns out (0x0000 is +0)."""
+    xb = _bf16_bits(x)
+    rows, cols = xb.shape
+    if axis == 1:
+        out = np.zeros((rows, padded_length(cols, blk)), dtype=np.uint16)
+    else:
+        out = np.zeros((padded_length(rows, blk), cols), dtype=np.uint16)
+    out[:rows, :cols] = xb
+    return out
+
+
 def rotate(x, blk: int, axis: int) -> np.ndarray:
     """Block-local rotation of a bf16 matrix.
 
     axis=1: along the contiguous dimension (blocks of ``blk`` consecutive
     elements of each row).  axis=0: along dimension 0 (blocks of ``blk``
-    consecutive rows of each column).  Returns fp64 of the same shape.
+    consecutive rows of each column).  Returns fp64 of the same shape.  A
+    rotated dimension that is not a multiple of blk is zero-padded first
+    (``pad_to_blocks``), and the result has the padded shape.
     """
     xb = _bf16_bits(x)
+    if (xb.shape[1] if axis == 1 else xb.shape[0]) % blk:
+        xb = pad_to_blocks(xb, blk, axis)
     rows, cols = xb.shape
     out = np.empty((rows, cols), dtype=np.float64)
     lib = _load()
@@ -145,8 +170,13 @@ def rotate_signed(x, blk: int, axis: int, signs) -> np.ndarray:
     """Random-sign rotation H (D x): each element times the +-1 sign of its
     position along the rotated dimension, then the block transform."""
     xb = _bf16_bits(x)
-    rows, cols = xb.shape
     sg = np.ascontiguousarray(signs, dtype=np.int8)
+    n = xb.shape[1] if axis == 1 else xb.shape[0]
+    if n % blk:
+        # padded positions hold zeros, whose sign does not matter
+        xb = pad_to_blocks(xb, blk, axis)
+        sg = np.concatenate([sg[:n], np.ones(padded_length(n, blk) - n, dtype=np.int8)])
+    rows, cols = xb.shape
     assert sg.shape == ((cols,) if axis == 1 else (rows,))
     out = np.empty((rows, cols), dtype=np.float64)
     lib = _load()
@@ -247,8 +277,11 @@ def dequant(acc: np.ndarray, sa: np.ndarray, sb: np.ndarray) -> np.ndarray:
 
 
 def linear_fwd(x, w, blk: int, qtype: int) -> np.ndarray:
-    """Y[M, N] = X W^T with both operands rotated along K and quantised per row."""
+    """Y[M, N] = X W^T with both operands rotated along K and quantised per row
+    (K not a multiple of blk: both zero-padded along K first)."""
     xb, wb = _bf16_bits(x), _bf16_bits(w)
+    if xb.shape[1] % blk:
+        xb, wb = pad_to_blocks(xb, blk, 1), pad_to_blocks(wb, blk, 1)
     m, k = xb.shape
     n, _ = wb.shape
     y = np.empty((m, n), dtype=np.float64)
@@ -257,8 +290,11 @@ def linear_fwd(x, w, blk: int, qtype: int) -> np.ndarray:
 
 
 def linear_bwd_dx(dy, w, blk: int, qtype: int) -> np.ndarray:
-    """dX[M, K] = dY W with both operands rotated along N."""
+    """dX[M, K] = dY W with both operands rotated along N (N not a multiple of
+    blk: dY's columns and W's rows zero-padded first)."""
     dyb, wb = _bf16_bits(dy), _bf16_bits(w)
+    if dyb.shape[1] % blk:
+        dyb, wb = pad_to_blocks(dyb, blk, 1), pad_to_blocks(wb, blk, 0)
     m, n = dyb.shape
     _, k = wb.shape
     dx = np.empty((m, k), dtype=np.float64)
@@ -267,8 +303,11 @@ def linear_bwd_dx(dy, w, blk: int, qtype: int) -> np.ndarray:
 
 
 def linear_bwd_dw(dy, x, blk: int, qtype: int) -> np.ndarray:
-    """dW[N, K] = dY^T X with both operands rotated along M (tokens)."""
+    """dW[N, K] = dY^T X with both operands rotated along M (tokens; M not a
+    multiple of blk: the rows of both zero-padded first)."""
     dyb, xb = _bf16_bits(dy), _bf16_bits(x)
+    if dyb.shape[0] % blk:
+        dyb, xb = pad_to_blocks(dyb, blk, 0), pad_to_blocks(xb, blk, 0)
     m, n = dyb.shape
     _, k = xb.shape
     dw = np.empty((n, k), dtype=np.float64)

@@ -439,3 +439,82 @@ def test_stochastic_rounding_is_unbiased():
     # round to nearest is biased on the same values; stochastic is not
     q_rne, _, _ = oracle.quantize(v[:1], 0, oracle.INT8)
     assert np.mean(np.abs(q_rne.view(np.int8)[0] - t[0])) > 4 * np.mean(np.abs(mean - t[0]))
+
+
+# ------------------------------------------------------------------ zero padding
+@pytest.mark.parametrize("blk", [128, 256])
+@pytest.mark.parametrize("axis,shape", [(1, (3, 300)), (1, (2, 5)), (0, (200, 3)), (0, (70, 2))])
+def test_padded_rotation_equals_dense_h_on_zero_extended_input(blk, axis, shape):
+    """A rotated length that is not a multiple of blk: the oracle's rotation
+    equals the dense normalised Sylvester matrix applied block by block to the
+    input extended with zeros (built here independently)."""
+    if axis == 0 and blk == 256:
+        pytest.skip("dimension-0 rotations use block 128")
+    rng = np.random.default_rng(sum(shape) + blk)
+    x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(torch.bfloat16)
+    xd = x.double().numpy()
+    rows, cols = shape
+    n = cols if axis == 1 else rows
+    n_pad = -(-n // blk) * blk
+    h = _sylvester_block(blk) / np.sqrt(blk)
+    if axis == 1:
+        ext = np.zeros((rows, n_pad))
+        ext[:, :cols] = xd
+        expect = np.concatenate([ext[:, b:b + blk] @ h.T for b in range(0, n_pad, blk)], axis=1)
+    else:
+        ext = np.zeros((n_pad, cols))
+        ext[:rows, :] = xd
+        expect = np.concatenate([h @ ext[b:b + blk, :] for b in range(0, n_pad, blk)], axis=0)
+    got = oracle.rotate(x, blk, axis)
+    assert got.shape == expect.shape
+    np.testing.assert_allclose(got, expect, rtol=1e-12, atol=1e-12 * np.abs(expect).max())
+
+
+def test_padded_linear_layers_within_quantisation_bound():
+    """fwd with K, dX with N, dW with M not multiples of 128: the results stay
+    within the worst-case quantisation bound around the exact unpadded
+    products (zero padding leaves every product unchanged; anything else in the
+    padded positions would not)."""
+    rng = np.random.default_rng(31)
+    m, n, k, blk = 200, 136, 328, 128
+    x = torch.from_numpy(rng.standard_normal((m, k)).astype(np.float32))
+    x[:, 3] *= 50
+    x = x.to(torch.bfloat16)
+    w = torch.from_numpy((0.02 * rng.standard_normal((n, k))).astype(np.float32)).to(torch.bfloat16)
+    dy = torch.from_numpy((1e-3 * rng.standard_normal((m, n))).astype(np.float32)).to(torch.bfloat16)
+    xd, wd, dyd = x.double().numpy(), w.double().numpy(), dy.double().numpy()
+
+    def check(got, exact, a, b):
+        _, sa, _ = oracle.quantize(a, 0, oracle.INT8)
+        _, sb, _ = oracle.quantize(b, 0, oracle.INT8)
+        assert got.shape == exact.shape
+        assert np.all(np.abs(got - exact) <= _bound(a, sa, b, sb, _int8_err) * (1 + 1e-9) + 1e-15)
+        assert np.max(np.abs(got - exact)) < 0.05 * np.max(np.abs(exact))
+
+    # Y = X W^T over K = 328 (padded to 384)
+    check(oracle.linear_fwd(x, w, blk, oracle.INT8), xd @ wd.T, oracle.rotate(x, blk, 1), oracle.rotate(w, blk, 1))
+    # dX = dY W over N = 136 (padded to 256)
+    check(oracle.linear_bwd_dx(dy, w, blk, oracle.INT8), dyd @ wd, oracle.rotate(dy, blk, 1),
+          np.ascontiguousarray(oracle.rotate(w, blk, 0).T))
+    # dW = dY^T X over M = 200 (padded to 256)
+    check(oracle.linear_bwd_dw(dy, x, blk, oracle.INT8), dyd.T @ xd,
+          np.ascontiguousarray(oracle.rotate(dy, blk, 0).T), np.ascontiguousarray(oracle.rotate(x, blk, 0).T))
+
+
+def test_padding_is_zero_not_garbage():
+    """A plausible mistake, planted on the CPU: padding with anything but zeros
+    breaks the product (the check above would fail on it)."""
+    rng = np.random.default_rng(32)
+    x = torch.from_numpy(rng.standard_normal((8, 200)).astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy(rng.standard_normal((6, 200)).astype(np.float32)).to(torch.bfloat16)
+    xp = oracle.pad_to_blocks(x, 128, 1)
+    assert xp.shape == (8, 256) and np.all(xp[:, 200:] == 0)
+    exact = x.double().numpy() @ w.double().numpy().T
+    xr, wr = oracle.rotate(x, 128, 1), oracle.rotate(w, 128, 1)
+    np.testing.assert_allclose(xr @ wr.T, exact, rtol=1e-10, atol=1e-10)
+    # ones in both operands' padding add 56 to every product
+    bad_x, bad_w = xp.copy(), oracle.pad_to_blocks(w, 128, 1)
+    bad_x[:, 200:] = _bf16_bits(torch.ones(8, 56, dtype=torch.bfloat16))
+    bad_w[:, 200:] = _bf16_bits(torch.ones(6, 56, dtype=torch.bfloat16))
+    bad = oracle.rotate(bad_x, 128, 1) @ oracle.rotate(bad_w, 128, 1).T
+    np.testing.assert_allclose(bad - exact, 56.0, rtol=1e-9)
