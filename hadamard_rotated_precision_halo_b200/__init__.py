@@ -131,16 +131,30 @@ def _out_dtype(otype: int):
     return torch.float32 if otype == HALO_OUT_FP32 else torch.bfloat16
 
 
+def padded_length(n: int, blk: int) -> int:
+    """A rotated dimension of n elements, zero-padded to whole blocks."""
+    return -(-n // blk) * blk
+
+
+def codes_shape(rows: int, cols: int, axis: int, blk: int):
+    """Shape of the codes: the rotated dimension zero-padded to whole blocks
+    (blocks of 128 rows along dimension 0)."""
+    if axis == HALO_AXIS_COLS:
+        return rows, padded_length(cols, blk)
+    return padded_length(rows, 128), cols
+
+
 def halo_hadamard_quantize(x: torch.Tensor, axis: int, blk: int, qtype: int, q_out=None, scales_out=None,
                            stream=None):
     """Rotate + quantise a bf16 [rows, cols] matrix; returns (codes, scales).
 
     axis HALO_AXIS_COLS: blocks along each row, one scale per row.
     axis HALO_AXIS_ROWS: blocks along dimension 0, one scale per column.
+    The codes cover the rotated dimension zero-padded to whole blocks.
     """
     rows, cols = x.shape
     if q_out is None:
-        q_out = torch.empty((rows, cols), dtype=_code_dtype(qtype), device=x.device)
+        q_out = torch.empty(codes_shape(rows, cols, axis, blk), dtype=_code_dtype(qtype), device=x.device)
     if scales_out is None:
         scales_out = torch.empty(rows if axis == HALO_AXIS_COLS else cols, dtype=torch.float32, device=x.device)
     st = lib().halo_hadamard_quantize(_ptr(x), rows, cols, x.stride(0), axis, blk, qtype, _ptr(q_out),
@@ -156,7 +170,7 @@ def halo_hadamard_quantize_ex(x: torch.Tensor, axis: int, blk: int, qtype: int, 
     (uint16 stored as int16/uint16 tensor of x's shape)."""
     rows, cols = x.shape
     if q_out is None:
-        q_out = torch.empty((rows, cols), dtype=_code_dtype(qtype), device=x.device)
+        q_out = torch.empty(codes_shape(rows, cols, axis, blk), dtype=_code_dtype(qtype), device=x.device)
     if scales_out is None:
         scales_out = torch.empty(rows if axis == HALO_AXIS_COLS else cols, dtype=torch.float32, device=x.device)
     ld_rand = rand_bits.stride(0) if rand_bits is not None else 0
@@ -172,10 +186,11 @@ def halo_hadamard_quantize_dual(x: torch.Tensor, blk: int, q_int8=None, scales_i
     """Rotate along the contiguous dim once, quantise to INT8 and to E4M3;
     returns (int8 codes, int8 scales, e4m3 codes, e4m3 scales)."""
     rows, cols = x.shape
+    shape = codes_shape(rows, cols, HALO_AXIS_COLS, blk)
     if q_int8 is None:
-        q_int8 = torch.empty((rows, cols), dtype=_code_dtype(HALO_Q_INT8), device=x.device)
+        q_int8 = torch.empty(shape, dtype=_code_dtype(HALO_Q_INT8), device=x.device)
     if q_e4m3 is None:
-        q_e4m3 = torch.empty((rows, cols), dtype=_code_dtype(HALO_Q_E4M3), device=x.device)
+        q_e4m3 = torch.empty(shape, dtype=_code_dtype(HALO_Q_E4M3), device=x.device)
     if scales_int8 is None:
         scales_int8 = torch.empty(rows, dtype=torch.float32, device=x.device)
     if scales_e4m3 is None:

@@ -65,21 +65,29 @@ cudaError_t set_smem_attr(K kernel, int optin) {
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
-typedef void (*RowsKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, RotqRowsParams);
+typedef void (*RowsKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           RotqRowsParams);
 typedef void (*Cols1Kernel)(const CUtensorMap, const CUtensorMap, RotqCols1Params);
 typedef void (*Cols2Kernel)(const CUtensorMap, const CUtensorMap, RotqColsParams);
 
 // `ext`: the instantiation that reads the variants' optional inputs (signs,
 // random bits); the plain path is compiled without them.
-// qtype kQtDual (2): INT8 and E4M3 codes from one read (plain path only).
-RowsKernel rows_kernel(int blk, int qtype, bool ext) {
-  if (qtype == kQtDual) return blk == 128 ? rotq_rows_kernel<128, kQtDual, 0> : rotq_rows_kernel<256, kQtDual, 0>;
+template <int PAD>
+RowsKernel rows_kernel_for(int blk, int qtype, bool ext) {
+  if (qtype == kQtDual)
+    return blk == 128 ? rotq_rows_kernel<128, kQtDual, 0, PAD> : rotq_rows_kernel<256, kQtDual, 0, PAD>;
   if (blk == 128) {
-    if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<128, 0, 1> : rotq_rows_kernel<128, 0, 0>;
-    return ext ? rotq_rows_kernel<128, 1, 1> : rotq_rows_kernel<128, 1, 0>;
+    if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<128, 0, 1, PAD> : rotq_rows_kernel<128, 0, 0, PAD>;
+    return ext ? rotq_rows_kernel<128, 1, 1, PAD> : rotq_rows_kernel<128, 1, 0, PAD>;
   }
-  if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<256, 0, 1> : rotq_rows_kernel<256, 0, 0>;
-  return ext ? rotq_rows_kernel<256, 1, 1> : rotq_rows_kernel<256, 1, 0>;
+  if (qtype == HALO_Q_INT8) return ext ? rotq_rows_kernel<256, 0, 1, PAD> : rotq_rows_kernel<256, 0, 0, PAD>;
+  return ext ? rotq_rows_kernel<256, 1, 1, PAD> : rotq_rows_kernel<256, 1, 0, PAD>;
+}
+
+// qtype kQtDual (2): INT8 and E4M3 codes from one read (plain path only).
+// pad: the row length is not a multiple of the block.
+RowsKernel rows_kernel(int blk, int qtype, bool ext, bool pad) {
+  return pad ? rows_kernel_for<1>(blk, qtype, ext) : rows_kernel_for<0>(blk, qtype, ext);
 }
 
 template <int QT, int EXT>
@@ -131,12 +139,18 @@ halo_status_t device_setup(int* dev_out) {
     }
     int optin = 0;
     HALO_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
-    HALO_CUDA(set_smem_attr(rows_kernel(128, kQtDual, false), optin));
-    HALO_CUDA(set_smem_attr(rows_kernel(256, kQtDual, false), optin));
+    for (int pad = 0; pad < 2; ++pad) {
+      HALO_CUDA(set_smem_attr(rows_kernel(128, kQtDual, false, pad), optin));
+      HALO_CUDA(set_smem_attr(rows_kernel(256, kQtDual, false, pad), optin));
+      for (int e = 0; e < 2; ++e) {
+        for (int qt = 0; qt < 2; ++qt) {
+          HALO_CUDA(set_smem_attr(rows_kernel(128, qt, e, pad), optin));
+          HALO_CUDA(set_smem_attr(rows_kernel(256, qt, e, pad), optin));
+        }
+      }
+    }
     for (int e = 0; e < 2; ++e) {
       for (int qt = 0; qt < 2; ++qt) {
-        HALO_CUDA(set_smem_attr(rows_kernel(128, qt, e), optin));
-        HALO_CUDA(set_smem_attr(rows_kernel(256, qt, e), optin));
         HALO_CUDA(set_smem_attr(cols_2pass_kernel(qt, e), optin));
         for (int nw = 1; nw <= 4; ++nw) {
           HALO_CUDA(set_smem_attr(cols_1pass_kernel(qt, nw, e), optin));
@@ -215,6 +229,9 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
   return HALO_OK;
 }
 
+// n rounded up to a multiple of b (the zero-padded length of a rotated dimension).
+int64_t pad_to(int64_t n, int64_t b) { return (n + b - 1) / b * b; }
+
 // ------------------------------------------------------------------------ rotq launches
 // qtype kQtDual: q / ld_q / scales take the INT8 output, q2 / ld_q2 / scales2
 // the E4M3 one (unused otherwise).
@@ -223,22 +240,39 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
                                cudaStream_t stream, int dev, void* q2 = nullptr, int64_t ld_q2 = 0,
                                float* scales2 = nullptr) {
   const bool dual = qtype == kQtDual;
-  const int nb = static_cast<int>(cols / 128);
+  // A row of `cols` elements is zero-padded to whole blocks: nb 128-element
+  // chunks, of which nbt are whole in the input and one more (tail > 0
+  // elements) is partial; chunks past that are all zero.
+  const int nb = static_cast<int>(pad_to(cols, blk) / 128);
+  const int nbt = static_cast<int>(cols / 128);
+  const int tail = static_cast<int>(cols % 128);
   // A row group of ceil(nb / 32) warps owns one row at a time; 4 warps per
   // CTA when a group fits in 4, else one group per CTA (up to 8 warps).
   const int gw = (nb + 31) / 32;
   const int groups = gw <= 4 ? 4 / gw : 1;
   const int threads = groups * gw * 32;
 
-  CUtensorMap tm_x, tm_q, tm_q2;
-  {
-    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
-    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(nb), 1};
-    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box,
+  CUtensorMap tm_x, tm_xt, tm_q, tm_q2;
+  if (tail) {
+    // The partial chunk: a 2-D view of X, one 128-element box per row.
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {128, 1};
+    halo_status_t st = encode(&tm_xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
                               CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != HALO_OK) return st;
   }
+  if (nbt > 0) {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nbt), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(nbt), 1};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  } else {
+    tm_x = tm_xt;  // never read: the kernel issues no 3-D load when nbt == 0
+  }
+  if (!tail) tm_xt = tm_x;  // never read
   {
     cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(ld_q)};
@@ -253,12 +287,15 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
       if (st != HALO_OK) return st;
     }
   }
-  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw, dual ? 2 : 1) + 128;  // + alignment slack
+  const bool pad = tail != 0 || nbt != nb;
+  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw, dual ? 2 : 1, pad) + 128;  // + alignment slack
 
   RotqRowsParams p;
   p.scales = scales;
   p.rows = rows;
   p.nb = nb;
+  p.nbt = nbt;
+  p.tail = tail;
   p.gw = gw;
   p.groups = groups;
   p.qmax = qtype == HALO_Q_E4M3 ? 448.f : 127.f;
@@ -267,14 +304,14 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   p.scales2 = scales2;
   p.scale_mult2 = static_cast<float>(1.0 / (448.0 * sqrt(static_cast<double>(blk))));
 
-  RowsKernel kern = rows_kernel(blk, qtype, ext);
+  RowsKernel kern = rows_kernel(blk, qtype, ext, pad);
   int per_sm = 0;
   HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
   if (per_sm < 1) per_sm = 1;
   const int64_t ctas_needed = (rows + groups - 1) / groups;
   const int grid = static_cast<int>(std::min<int64_t>(ctas_needed, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
   Launch L(dim3(grid), dim3(threads), smem, stream, 0);
-  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, tm_q2, p));
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_xt, tm_q, tm_q2, p));
   return HALO_OK;
 }
 
@@ -294,7 +331,7 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
     if (st != HALO_OK) return st;
   }
   {
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(pad_to(rows, 128))};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
     cuuint32_t box[2] = {kColsStrip, 128};
     halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
@@ -325,7 +362,9 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
 halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
                                int64_t ld_q, float* scales, const RotqExtras& ex, bool ext, cudaStream_t stream,
                                int dev) {
-  const int nblocks = static_cast<int>(rows / 128);
+  // Rows past the input (zero padding to whole 128-row blocks) are outside the
+  // input tensor map and arrive as zeros; the codes cover the padded rows.
+  const int nblocks = static_cast<int>(pad_to(rows, 128) / 128);
   // Most warps per CTA (up to 4) with at most 16 CTAs per cluster.
   for (int nw = 4; nw >= 1; --nw) {
     if (nblocks % nw == 0 && nblocks / nw <= 16)
@@ -348,7 +387,7 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
     if (st != HALO_OK) return st;
   }
   {
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(pad_to(rows, 128))};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
     cuuint32_t box[2] = {kColsStrip, 128};
     halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
@@ -467,18 +506,21 @@ halo_status_t check_hadamard_quantize(const void* x, int64_t rows, int64_t cols,
   if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
   if (axis == HALO_AXIS_ROWS && blk != 128) return HALO_ERR_BLOCK;
   if (rows <= 0 || cols <= 0 || ld_x < cols || ld_q < cols) return HALO_ERR_SHAPE;
-  if (axis == HALO_AXIS_COLS && (cols % blk != 0 || cols > 32768)) return HALO_ERR_SHAPE;
-  if (axis == HALO_AXIS_ROWS && (rows % blk != 0 || cols % 8 != 0)) return HALO_ERR_SHAPE;
+  // A rotated length that is not a multiple of blk is zero-padded; the codes
+  // cover the padded length.
+  if (axis == HALO_AXIS_COLS && (pad_to(cols, blk) > 32768 || ld_q < pad_to(cols, blk))) return HALO_ERR_SHAPE;
+  if (axis == HALO_AXIS_ROWS && cols % 8 != 0) return HALO_ERR_SHAPE;
   if (rows > (int64_t(1) << 31) - 1 || cols > (int64_t(1) << 31) - 1) return HALO_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(q) || !aligned16(scales) || (ld_x * 2) % 16 != 0 || ld_q % 16 != 0)
     return HALO_ERR_ALIGN;
   return HALO_OK;
 }
 
-halo_status_t check_extras(const int8_t* signs, const uint16_t* rand_bits, int64_t ld_rand, int64_t cols) {
+halo_status_t check_extras(const int8_t* signs, const uint16_t* rand_bits, int64_t ld_rand, int64_t cols,
+                           int axis, int blk) {
   if (signs && !aligned16(signs)) return HALO_ERR_ALIGN;
   if (rand_bits) {
-    if (ld_rand < cols) return HALO_ERR_SHAPE;
+    if (ld_rand < (axis == HALO_AXIS_COLS ? pad_to(cols, blk) : cols)) return HALO_ERR_SHAPE;
     if (!aligned16(rand_bits) || (ld_rand * 2) % 16 != 0) return HALO_ERR_ALIGN;
   }
   return HALO_OK;
@@ -513,23 +555,28 @@ struct WsLayout {
   size_t total;
 };
 
-WsLayout ws_layout(int64_t m, int64_t n, int64_t k, int which) {
+// Scratch of the linear layers: codes and scales of both operands of each GEMM,
+// the contraction dimension zero-padded to whole blocks (fwd: K to blk; dX: N
+// to 128; dW: M to 128).
+WsLayout ws_layout(int64_t m, int64_t n, int64_t k, int which, int blk) {
   WsLayout L = {};
   size_t sizes[8];
   int cnt;
   if (which == 0) {
-    sizes[0] = size_t(m) * k;
-    sizes[1] = size_t(n) * k;
+    const int64_t kp = pad_to(k, blk);
+    sizes[0] = size_t(m) * kp;
+    sizes[1] = size_t(n) * kp;
     sizes[2] = size_t(m) * 4;
     sizes[3] = size_t(n) * 4;
     cnt = 4;
   } else {
-    sizes[0] = size_t(m) * n;
-    sizes[1] = size_t(n) * k;
+    const int64_t np = pad_to(n, 128), mp = pad_to(m, 128);
+    sizes[0] = size_t(m) * np;
+    sizes[1] = size_t(np) * k;
     sizes[2] = size_t(m) * 4;
     sizes[3] = size_t(k) * 4;
-    sizes[4] = size_t(m) * n;
-    sizes[5] = size_t(m) * k;
+    sizes[4] = size_t(mp) * n;
+    sizes[5] = size_t(mp) * k;
     sizes[6] = size_t(n) * 4;
     sizes[7] = size_t(k) * 4;
     cnt = 8;
@@ -578,7 +625,8 @@ halo_status_t halo_device_error(int* where) {
 
 size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which) {
   if (m <= 0 || n <= 0 || k <= 0 || (which != 0 && which != 1)) return 0;
-  return ws_layout(m, n, k, which).total;
+  // forward: enough for either block size (K padded to 256 is the larger)
+  return ws_layout(m, n, k, which, which == 0 ? 256 : 128).total;
 }
 
 halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int axis,
@@ -587,7 +635,7 @@ halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_
                                         void* stream) {
   halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, axis, blk, qtype, q_out, ld_q, scales_out);
   if (st != HALO_OK) return st;
-  if ((st = check_extras(signs, rand_bits, ld_rand, cols)) != HALO_OK) return st;
+  if ((st = check_extras(signs, rand_bits, ld_rand, cols, axis, blk)) != HALO_OK) return st;
   int dev = 0;
   st = device_setup(&dev);
   if (st != HALO_OK) return st;
@@ -646,22 +694,24 @@ halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m,
   if (!x_bf16 || !w_bf16 || !y) return HALO_ERR_NULL;
   if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
   if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
-  if (m <= 0 || n <= 0 || k <= 0 || k % blk != 0 || k > 32768) return HALO_ERR_SHAPE;
+  if (m <= 0 || n <= 0 || k <= 0 || pad_to(k, blk) > 32768) return HALO_ERR_SHAPE;
   if (!ws) return HALO_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(m, n, k, 0);
+  const WsLayout L = ws_layout(m, n, k, 0, blk);
   if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
   const int64_t esz = otype == HALO_OUT_FP32 ? 4 : 2;
-  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y) || !aligned16(ws) || (n * esz) % 16 != 0)
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y) || !aligned16(ws) || (n * esz) % 16 != 0 ||
+      k % 8 != 0)
     return HALO_ERR_ALIGN;
+  const int64_t kp = pad_to(k, blk);  // K zero-padded to whole blocks
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   uint8_t* xq = w8 + L.off[0];
   uint8_t* wq = w8 + L.off[1];
   float* sx = reinterpret_cast<float*>(w8 + L.off[2]);
   float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
   halo_status_t st;
-  if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_COLS, blk, qtype, xq, k, sx, stream)) != HALO_OK) return st;
-  if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_COLS, blk, qtype, wq, k, sw, stream)) != HALO_OK) return st;
-  return halo_qgemm(xq, sx, HALO_MAJOR_K, k, wq, sw, HALO_MAJOR_K, k, m, n, k, qtype, y, otype, n, stream);
+  if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_COLS, blk, qtype, xq, kp, sx, stream)) != HALO_OK) return st;
+  if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_COLS, blk, qtype, wq, kp, sw, stream)) != HALO_OK) return st;
+  return halo_qgemm(xq, sx, HALO_MAJOR_K, kp, wq, sw, HALO_MAJOR_K, kp, m, n, kp, qtype, y, otype, n, stream);
 }
 
 halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k,
@@ -671,8 +721,8 @@ halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, in
   if (!x_bf16 || !w_bf16 || !y) return HALO_ERR_NULL;
   if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
   if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
-  if (m <= 0 || n <= 0 || k <= 0 || k % blk != 0 || k > 32768) return HALO_ERR_SHAPE;
-  const size_t need = ws_layout(m, n, k, 0).total;
+  if (m <= 0 || n <= 0 || k <= 0 || pad_to(k, blk) > 32768) return HALO_ERR_SHAPE;
+  const size_t need = ws_layout(m, n, k, 0, blk).total;
   if (need > HALO_NOALLOC_SCRATCH_BYTES) {
     snprintf(g_last_detail, sizeof g_last_detail,
              "halo_linear_fwd_noalloc: these sizes need %zu bytes of scratch, the library's static array holds %llu",
@@ -696,15 +746,16 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
   if (!valid_qtype(qtype) || (dx && !valid_otype(otype_dx)) || (dw && !valid_otype(otype_dw))) return HALO_ERR_DTYPE;
   if (blk != 128) return HALO_ERR_BLOCK;
   if (m <= 0 || n <= 0 || k <= 0) return HALO_ERR_SHAPE;
-  if (dx && (n % blk != 0 || n > 32768 || k % 16 != 0)) return HALO_ERR_SHAPE;
-  if (dw && (m % blk != 0 || n % 16 != 0 || k % 16 != 0)) return HALO_ERR_SHAPE;
+  if (dx && (pad_to(n, blk) > 32768 || k % 16 != 0)) return HALO_ERR_SHAPE;
+  if (dw && (n % 16 != 0 || k % 16 != 0)) return HALO_ERR_SHAPE;
   if (!ws) return HALO_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(m, n, k, 1);
+  const WsLayout L = ws_layout(m, n, k, 1, blk);
   if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
   if (!aligned16(dy_bf16) || (x_bf16 && !aligned16(x_bf16)) || (w_bf16 && !aligned16(w_bf16)) ||
       (dx && !aligned16(dx)) || (dw && !aligned16(dw)) || !aligned16(ws))
     return HALO_ERR_ALIGN;
   if (dx && (k * (otype_dx == HALO_OUT_FP32 ? 4 : 2)) % 16 != 0) return HALO_ERR_ALIGN;
+  if (n % 8 != 0) return HALO_ERR_ALIGN;  // dY's rows: a multiple of 16 bytes
   if (dw && (k * (otype_dw == HALO_OUT_FP32 ? 4 : 2)) % 16 != 0) return HALO_ERR_ALIGN;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   halo_status_t st;
@@ -713,12 +764,13 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
     uint8_t* wq = w8 + L.off[1];
     float* sdy = reinterpret_cast<float*>(w8 + L.off[2]);
     float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
-    // dX[M,K] = dY[M,N] W[N,K]: contraction over N.
-    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, qtype, dyq, n, sdy, stream)) != HALO_OK)
+    // dX[M,K] = dY[M,N] W[N,K]: contraction over N (zero-padded to np).
+    const int64_t np = pad_to(n, blk);
+    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, qtype, dyq, np, sdy, stream)) != HALO_OK)
       return st;
     if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_ROWS, blk, qtype, wq, k, sw, stream)) != HALO_OK)
       return st;
-    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_K, n, wq, sw, HALO_MAJOR_MN, k, m, k, n, qtype, dx, otype_dx, k,
+    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_K, np, wq, sw, HALO_MAJOR_MN, k, m, k, np, qtype, dx, otype_dx, k,
                          stream)) != HALO_OK)
       return st;
   }
@@ -727,12 +779,13 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
     uint8_t* xq = w8 + L.off[5];
     float* sdy = reinterpret_cast<float*>(w8 + L.off[6]);
     float* sx = reinterpret_cast<float*>(w8 + L.off[7]);
-    // dW[N,K] = dY^T[N,M] X[M,K]: contraction over M (tokens).
+    // dW[N,K] = dY^T[N,M] X[M,K]: contraction over M (tokens, zero-padded to mp).
+    const int64_t mp = pad_to(m, blk);
     if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, qtype, dyq, n, sdy, stream)) != HALO_OK)
       return st;
     if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_ROWS, blk, qtype, xq, k, sx, stream)) != HALO_OK)
       return st;
-    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_MN, n, xq, sx, HALO_MAJOR_MN, k, n, k, m, qtype, dw, otype_dw, k,
+    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_MN, n, xq, sx, HALO_MAJOR_MN, k, n, k, mp, qtype, dw, otype_dw, k,
                          stream)) != HALO_OK)
       return st;
   }

@@ -193,7 +193,9 @@ __device__ __forceinline__ float rand_unit(uint32_t bits16) { return static_cast
 struct RotqRowsParams {
   float* scales;
   int64_t rows;
-  int nb;        // 128-element chunks per row (cols / 128)
+  int nb;        // 128-element chunks per padded row (cols rounded up to the block, / 128)
+  int nbt;       // whole 128-element chunks of the input row (loaded by the 3-D TMA view)
+  int tail;      // elements of the input's last, partial chunk (0: none; loaded by a 2-D TMA box)
   int gw;        // warps per row group
   int groups;    // row groups per CTA
   float qmax;
@@ -207,12 +209,14 @@ struct RotqRowsParams {
 // scales through tm_q / scales, E4M3 codes with theirs through tm_q2 / scales2.
 constexpr int kQtDual = 2;
 
-// Shared-memory bytes of one row group: 2 input stages and one code tile (two
-// for the dual output).
-__host__ __device__ inline uint32_t rows_group_in_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsInSlot; }
+// Shared-memory bytes of one row group: 2 input stages (the per-thread slots,
+// then, when padding, 256 bytes for a partial last chunk) and one code tile
+// (two for the dual output).
+__host__ __device__ inline uint32_t rows_group_slots_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsInSlot; }
+__host__ __device__ inline uint32_t rows_group_in_bytes(int gw, int pad) { return rows_group_slots_bytes(gw) + (pad ? 256 : 0); }
 __host__ __device__ inline uint32_t rows_group_out_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsOutSlot; }
-__host__ __device__ inline uint32_t rows_group_smem(int gw, int ntiles = 1) {
-  return 2 * rows_group_in_bytes(gw) + ntiles * rows_group_out_bytes(gw);
+__host__ __device__ inline uint32_t rows_group_smem(int gw, int ntiles, int pad) {
+  return 2 * rows_group_in_bytes(gw, pad) + ntiles * rows_group_out_bytes(gw);
 }
 
 __device__ __forceinline__ void group_sync(int gw, int grp) {
@@ -222,10 +226,13 @@ __device__ __forceinline__ void group_sync(int gw, int grp) {
     named_bar_sync(1 + grp, gw * 32);
 }
 
-template <int BLK, int QT, int EXT>
+// PAD = 1: the row length is not a multiple of the block (zero padding); the
+// instantiation for whole blocks (PAD = 0) carries none of that logic.
+template <int BLK, int QT, int EXT, int PAD>
 __global__ void __launch_bounds__(256)
-    rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_q2, RotqRowsParams p) {
+    rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xt,
+                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
+                     RotqRowsParams p) {
   constexpr int kTiles = QT == kQtDual ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -239,10 +246,14 @@ __global__ void __launch_bounds__(256)
   const int wig = warp - grp * gw;          // warp index inside the group
   const int chunk = wig * 32 + lane;        // this thread's 128-element chunk of the row
   const bool is_active = chunk < p.nb;
+  // Chunks past the input (zero padding up to the block) hold zeros.
+  const bool is_zero = PAD && (chunk > p.nbt || (chunk == p.nbt && p.tail == 0));
   const bool leader = (wig == 0 && lane == 0);
-  const uint32_t in_bytes = static_cast<uint32_t>(p.nb) * kRowsInSlot;  // one row's box
-  uint8_t* g_in = smem + grp * rows_group_smem(gw, kTiles);
-  uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw);
+  // One row: the 3-D box of whole chunks, plus the partial chunk's 2-D box.
+  const uint32_t in_bytes = PAD ? static_cast<uint32_t>(p.nbt) * kRowsInSlot + (p.tail ? 256u : 0u)
+                               : static_cast<uint32_t>(p.nb) * kRowsInSlot;
+  uint8_t* g_in = smem + grp * rows_group_smem(gw, kTiles, PAD);
+  uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw, PAD);
   uint8_t* g_out2 = g_out + rows_group_out_bytes(gw);  // QT = 2 only
 
   if (leader) {
@@ -250,6 +261,7 @@ __global__ void __launch_bounds__(256)
     mbar_init(&full_bar[grp][1], 1);
     fence_mbar_init();
     prefetch_tmap(&tm_x);
+    if (PAD && p.tail) prefetch_tmap(&tm_xt);
     prefetch_tmap(&tm_q);
     if (QT == kQtDual) prefetch_tmap(&tm_q2);
   }
@@ -263,9 +275,13 @@ __global__ void __launch_bounds__(256)
 
   auto issue = [&](int64_t it) {
     const int st = static_cast<int>(it & 1);
+    const int32_t row = static_cast<int32_t>(first + it * step);
+    uint8_t* dst = g_in + st * rows_group_in_bytes(gw, PAD);
     mbar_arrive_expect_tx(&full_bar[grp][st], in_bytes);
-    tma_load_3d(g_in + st * rows_group_in_bytes(gw), &tm_x, &full_bar[grp][st], 0, 0,
-                static_cast<int32_t>(first + it * step));
+    if (!PAD || p.nbt > 0) tma_load_3d(dst, &tm_x, &full_bar[grp][st], 0, 0, row);
+    // Partial last chunk: elements past the row's end are out of the 2-D
+    // tensor and arrive as zeros (the zero padding).
+    if (PAD && p.tail) tma_load_2d(dst + rows_group_slots_bytes(gw), &tm_xt, &full_bar[grp][st], p.nbt * 128, row);
   };
   if (leader) {
     if (nmine > 0) issue(0);
@@ -282,8 +298,10 @@ __global__ void __launch_bounds__(256)
       dead = !ok;
     }
     float2 v[64];
-    if (is_active && !dead) {
-      const uint4* src = reinterpret_cast<const uint4*>(g_in + st * rows_group_in_bytes(gw) + chunk * kRowsInSlot);
+    if (is_active && !is_zero && !dead) {
+      const uint8_t* stage = g_in + st * rows_group_in_bytes(gw, PAD);
+      const uint4* src = reinterpret_cast<const uint4*>(!PAD || chunk < p.nbt ? stage + chunk * kRowsInSlot
+                                                                              : stage + rows_group_slots_bytes(gw));
       const uint4* sgn = reinterpret_cast<const uint4*>(p.ex.signs + static_cast<int64_t>(chunk) * 128);
 #pragma unroll
       for (int k = 0; k < 16; ++k) {

@@ -51,8 +51,8 @@ extern "C" {
 typedef enum {
   HALO_OK = 0,
   HALO_ERR_NULL = 1,        /* a required pointer is NULL                      */
-  HALO_ERR_SHAPE = 2,       /* a size <= 0, a dimension not a multiple of blk, */
-                            /* or a size beyond a documented limit             */
+  HALO_ERR_SHAPE = 2,       /* a size <= 0, a stride shorter than its row, or  */
+                            /* a size beyond a documented limit                */
   HALO_ERR_BLOCK = 3,       /* blk not supported for this call                 */
   HALO_ERR_ALIGN = 4,       /* pointer not 16-byte aligned / stride rule       */
   HALO_ERR_DTYPE = 5,       /* unknown qtype / otype / axis / major            */
@@ -80,18 +80,25 @@ typedef enum {
 } halo_major_t;
 
 /*
- * Rotate + quantise one bf16 matrix X[rows, cols] (row stride ld_x elements).
- *   axis = HALO_AXIS_COLS: cols % blk == 0, blk in {128, 256}, cols <= 32768.
- *       scales_out[rows]:  s_r = max_c |Xrot[r, c]| / qmax.
- *   axis = HALO_AXIS_ROWS: rows % blk == 0, blk == 128, cols % 8 == 0.
- *       scales_out[cols]:  s_c = max_r |Xrot[r, c]| / qmax.
- * Xrot is X with every block transformed by H_blk / sqrt(blk).  q_out[rows,
- * cols] (row stride ld_q bytes) receives q = round-half-even(Xrot / s)
- * clamped to +-127 as two's-complement int8 (qtype INT8), or Xrot / s rounded
- * to nearest-even and saturated to +-448 as OCP E4M3 bytes (qtype E4M3).  A
- * group whose max is 0 gets scale 0 and all-zero codes.  The codes keep the
- * input's layout in both axes (nothing is transposed); halo_qgemm reads the
- * dimension-0-rotated codes as an MN-major operand.
+ * Rotate + quantise one bf16 matrix X[rows, cols] (row stride ld_x elements,
+ * ld_x * 2 a multiple of 16 bytes).
+ *   axis = HALO_AXIS_COLS: blk in {128, 256}; cols_p = cols rounded up to a
+ *       multiple of blk, cols_p <= 32768.  Codes q_out[rows, cols_p], ld_q >=
+ *       cols_p.  scales_out[rows]: s_r = max_c |Xrot[r, c]| / qmax.
+ *   axis = HALO_AXIS_ROWS: blk == 128, cols % 8 == 0; rows_p = rows rounded
+ *       up to a multiple of 128.  Codes q_out[rows_p, cols] (the buffer must
+ *       hold rows_p rows of ld_q bytes).  scales_out[cols]: s_c = max_r
+ *       |Xrot[r, c]| / qmax.
+ * A rotated length that is not a multiple of the block is zero-padded to
+ * whole blocks (QWHA page, sec. 3.1 and 5: zero-fill to the transform
+ * length); the codes cover the padded length.  Xrot is the (padded) X with
+ * every block transformed by H_blk / sqrt(blk).  q_out (row stride ld_q bytes,
+ * a multiple of 16) receives q = round-half-even(Xrot / s) clamped to +-127 as
+ * two's-complement int8 (qtype INT8), or Xrot / s rounded to nearest-even and
+ * saturated to +-448 as OCP E4M3 bytes (qtype E4M3).  A group whose max is 0
+ * gets scale 0 and all-zero codes.  The codes keep the input's layout in both
+ * axes (nothing is transposed); halo_qgemm reads the dimension-0-rotated codes
+ * as an MN-major operand.
  * Defined by: HALO paper page (abstract; "key design": INT8 or FP8); QWHA page
  * sec. 2.1-2.2 (Walsh-Hadamard transform, symmetric quantiser).
  */
@@ -102,16 +109,18 @@ halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t c
 /*
  * halo_hadamard_quantize with the two variants of the rotation and rounding:
  *   signs      NULL, or int8 +1 / -1 (only the sign bit is read) for every
- *              position along the rotated dimension (`cols` entries for
- *              HALO_AXIS_COLS, `rows` for HALO_AXIS_ROWS), 16-byte aligned:
+ *              position along the rotated dimension, padded length (cols_p
+ *              entries for HALO_AXIS_COLS, rows_p for HALO_AXIS_ROWS; the
+ *              entries past the input meet zeros), 16-byte aligned:
  *              random-sign rotation, each block becomes H_blk D x / sqrt(blk)
  *              with D = diag(signs).  Both operands of a GEMM must use the
  *              same signs along the contraction dimension; the product is
  *              then unchanged, since (H D)^T (H D) = I.  Seeded random signs
  *              shared by all workers: HALO blog page, sec. 4.2.
- *   rand_bits  NULL (round half to even), or 16 random bits per element,
- *              layout [rows, cols] with row stride ld_rand elements (16-byte
- *              aligned base, ld_rand * 2 a multiple of 16): stochastic
+ *   rand_bits  NULL (round half to even), or 16 random bits per element of
+ *              the codes, layout [rows, cols_p] (HALO_AXIS_COLS) or [rows_p,
+ *              cols] (HALO_AXIS_ROWS) with row stride ld_rand elements
+ *              (16-byte aligned base, ld_rand * 2 a multiple of 16): stochastic
  *              rounding.  With u = rand_bits / 65536, t = Xrot / s rounds to
  *              its upper grid neighbour when u < (t - lo) / (hi - lo), else
  *              to its lower one (INT8 grid clamped to +-127; E4M3 grid
@@ -126,7 +135,7 @@ halo_status_t halo_hadamard_quantize_ex(const void* x_bf16, int64_t rows, int64_
 /*
  * Both 8-bit encodings of one rotation from a single read of X: the block
  * rotation along the contiguous dimension (HALO_AXIS_COLS) of
- * halo_hadamard_quantize, quantised per row to INT8 (codes q_int8 [rows, cols],
+ * halo_hadamard_quantize, quantised per row to INT8 (codes q_int8 [rows, cols_p],
  * row stride ld_q8 bytes, scales_int8 [rows] = amax / (127 sqrt(blk))) and to
  * E4M3 (q_e4m3, ld_qf8, scales_e4m3 [rows] = amax / (448 sqrt(blk))).  Each
  * output equals what halo_hadamard_quantize writes for its qtype, byte for
@@ -160,15 +169,18 @@ halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t
 
 /*
  * Scratch bytes halo_linear_fwd (which = 0) or halo_linear_bwd (which = 1)
- * needs for these sizes: the operands' codes and scales.
+ * needs for these sizes: the operands' codes (contraction dimension
+ * zero-padded to whole blocks; the forward size covers either block size) and
+ * scales.
  */
 size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which);
 
 /*
  * Forward linear layer Y[M, N] = X[M, K] W[N, K]^T with both operands
- * rotated along K (blocks of blk, K % blk == 0), quantised per row (qtype),
- * multiplied on codes and dequantised.  x, w, y dense row-major.  ws must hold
- * halo_workspace_size(m, n, k, 0) bytes and be 16-byte aligned.
+ * rotated along K (blocks of blk; K % 8 == 0; a K that is not a multiple of
+ * blk is zero-padded to whole blocks, at most 32768), quantised per row
+ * (qtype), multiplied on codes and dequantised.  x, w, y dense row-major.  ws
+ * must hold halo_workspace_size(m, n, k, 0) bytes and be 16-byte aligned.
  * Defined by: HALO paper page, abstract (rotations in the forward pass).
  */
 halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
@@ -178,9 +190,11 @@ halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m,
 /*
  * Backward linear layer for Y = X W^T, given dY[M, N], X[M, K], W[N, K]:
  *   dX[M, K] = dY W:    dY rotated along N per row, W rotated along N
- *                       (dimension 0) per column; requires N % blk == 0.
+ *                       (dimension 0) per column; K % 16 == 0.
  *   dW[N, K] = dY^T X:  dY and X both rotated along M (dimension 0), one
- *                       scale per column; requires M % blk == 0.
+ *                       scale per column; N % 16 == 0, K % 16 == 0.
+ * N % 8 == 0.  An N (dX) or M (dW) that is not a multiple of blk is
+ * zero-padded to whole blocks (N padded at most 32768).
  * blk must be 128.  dx or dw may be NULL to skip that product (the inputs it
  * alone needs may then be NULL too).  All matrices dense row-major.  ws must
  * hold halo_workspace_size(m, n, k, 1) bytes.

@@ -65,6 +65,8 @@ def test_workspace_size(lib):
     m, n, k = 1024, 512, 768
     fwd = lib.halo_workspace_size(m, n, k, 0)
     assert fwd >= m * k + n * k + 4 * (m + n)
+    # zero padding of the contraction dimension: K = 700 needs codes for 768 (block 256)
+    assert lib.halo_workspace_size(m, n, 700, 0) >= (m + n) * 768 + 4 * (m + n)
     bwd = lib.halo_workspace_size(m, n, k, 1)
     assert bwd >= 2 * m * n + n * k + m * k + 4 * (m + 2 * n + k)
     assert lib.halo_workspace_size(0, n, k, 0) == 0
@@ -82,10 +84,11 @@ def test_hadamard_quantize_host_validation(lib):
     assert _hq(lib, axis=3) == DTYPE
     assert _hq(lib, blk=64) == BLOCK
     assert _hq(lib, axis=1, blk=256) == BLOCK
-    assert _hq(lib, cols=500, ld_x=512, ld_q=512) == SHAPE       # not a multiple of blk
+    assert _hq(lib, cols=500, ld_x=512, ld_q=504) == SHAPE       # codes need the zero-padded length (512)
     assert _hq(lib, rows=0) == SHAPE
     assert _hq(lib, cols=65536, ld_x=65536, ld_q=65536) == SHAPE  # beyond the row-kernel limit
-    assert _hq(lib, axis=1, rows=200) == SHAPE                    # rows % 128
+    assert _hq(lib, cols=32770, ld_x=32776, ld_q=32896) == SHAPE  # padded row beyond 32768
+    assert _hq(lib, axis=1, cols=500, ld_x=504, ld_q=512) == SHAPE  # dim-0 rotation: cols % 8
     assert _hq(lib, ld_x=256) == SHAPE                            # ld < cols
     assert _hq(lib, x=MISALIGNED) == ALIGN
     assert _hq(lib, ld_x=516, ld_q=516) == ALIGN                  # bf16 row stride not 16 B
@@ -115,7 +118,9 @@ def test_linear_host_validation(lib):
     f = lib.halo_linear_fwd
     assert f(None, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, ws, None) == NULL
     assert f(FAKE, FAKE, 256, 256, 512, 64, 0, FAKE, 0, FAKE, ws, None) == BLOCK
-    assert f(FAKE, FAKE, 256, 256, 500, 128, 0, FAKE, 0, FAKE, ws, None) == SHAPE
+    assert f(FAKE, FAKE, 256, 256, 500, 128, 0, FAKE, 0, FAKE, ws, None) == ALIGN     # 1000-byte rows of X
+    assert f(FAKE, FAKE, 256, 256, 32776, 128, 0, FAKE, 0, FAKE, ws, None) == SHAPE   # K padded beyond 32768
+    assert f(FAKE, FAKE, 256, 256, 520, 128, 0, FAKE, 0, FAKE, ws, None) == WORKSPACE  # K padded to 640
     assert f(FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, None, ws, None) == WORKSPACE
     assert f(FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, ws - 1, None) == WORKSPACE
     assert f(FAKE, FAKE, 256, 256, 512, 128, 9, FAKE, 0, FAKE, ws, None) == DTYPE
@@ -124,7 +129,8 @@ def test_linear_host_validation(lib):
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, None, 0, None, 0, FAKE, wsb, None) == NULL
     assert b(FAKE, None, FAKE, 256, 256, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == NULL  # dW needs X
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 256, 0, FAKE, 0, FAKE, 0, FAKE, wsb, None) == BLOCK
-    assert b(FAKE, FAKE, FAKE, 200, 256, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == SHAPE  # M % 128
+    assert b(FAKE, FAKE, FAKE, 256, 200, 512, 128, 0, None, 0, FAKE, 0, FAKE, wsb, None) == SHAPE  # dW: N % 16
+    assert b(FAKE, FAKE, FAKE, 256, 300, 512, 128, 0, FAKE, 0, None, 0, FAKE, wsb, None) == WORKSPACE  # N pads to 384
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE
 
 
@@ -152,6 +158,6 @@ def test_hadamard_quantize_dual_host_validation(lib):
     assert call(a5=None) == NULL        # INT8 codes
     assert call(a10=None) == NULL       # E4M3 scales
     assert call(a4=64) == BLOCK
-    assert call(a2=500, a3=512) == SHAPE
+    assert call(a2=500, a3=512, a6=504) == SHAPE   # INT8 codes shorter than the padded row (512)
     assert call(a8=MISALIGNED) == ALIGN
     assert call(a9=520) == ALIGN        # E4M3 row stride not a multiple of 16

@@ -13,7 +13,7 @@ import torch
 import hadamard_rotated_precision_halo_b200 as halo
 import oracle
 from hadamard_rotated_precision_halo_b200 import inputs
-from tests._parity import check_codes, check_output, oracle_operand
+from tests._parity import check_codes, check_codes_stochastic, check_output, oracle_operand
 
 pytestmark = pytest.mark.gpu
 
@@ -379,6 +379,87 @@ def test_rotq_dual_full_size_16384x4096():
     for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
         codes, scales, t = oracle_operand(xs, 1, 128, qt)
         check_codes(q[rows], s[rows], codes, scales, t, qt)
+
+
+# ------------------------------------------------------------ zero padding (ragged lengths)
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols,blk", [(37, 1000, 128), (5, 296, 256), (9, 72, 128), (3, 200, 256),
+                                           (4, 32760, 128), (6, 384, 256)])
+def test_rotq_rows_padded_parity(qtype, rows, cols, blk):
+    """Row length not a multiple of blk: the partial chunk arrives by its own
+    TMA box (zeros past the row), whole padding chunks are zeros; the codes
+    cover the padded length."""
+    x = inputs.activations(rows, cols, seed=rows * 3 + cols, device="cpu")
+    q, s = halo.halo_hadamard_quantize(_cuda(x), COLS, blk, qtype)
+    torch.cuda.synchronize()
+    assert tuple(q.shape) == (rows, halo.padded_length(cols, blk))
+    codes, scales, t = oracle_operand(x, 1, blk, qtype)
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols", [(1000, 48), (200, 64), (70, 32), (130, 80), (8300, 16), (28700, 16)])
+def test_rotq_cols_padded_parity(qtype, rows, cols):
+    """Column length not a multiple of 128 (one-pass and two-pass kernels): rows
+    past the input read as zeros; the codes cover the padded rows."""
+    x = inputs.activations(rows, cols, seed=rows + 5 * cols, device="cpu")
+    q, s = halo.halo_hadamard_quantize(_cuda(x), ROWS, 128, qtype)
+    torch.cuda.synchronize()
+    assert tuple(q.shape) == (halo.padded_length(rows, 128), cols)
+    codes, scales, t = oracle_operand(x, 0, 128, qtype)
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+def test_rotq_dual_padded_parity():
+    x = inputs.activations(7, 1000, seed=77, device="cpu")
+    q8, s8, qf, sf = halo.halo_hadamard_quantize_dual(_cuda(x), 128)
+    torch.cuda.synchronize()
+    for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
+        codes, scales, t = oracle_operand(x, 1, 128, qt)
+        check_codes(q, s, codes, scales, t, qt)
+
+
+@pytest.mark.parametrize("axis,rows,cols", [(COLS, 37, 1000), (ROWS, 1000, 48)])
+def test_padded_variants_parity(axis, rows, cols):
+    """Signs and random bits cover the padded length (their padded entries meet
+    zeros and change nothing)."""
+    x = inputs.activations(rows, cols, seed=91, device="cpu")
+    n = cols if axis == COLS else rows
+    npad = halo.padded_length(n, 128)
+    s = _signs_t(npad, seed=92)
+    shape = (rows, npad) if axis == COLS else (npad, cols)
+    rb = _rand_bits(*shape, seed=93)
+    q, sc = halo.halo_hadamard_quantize_ex(_cuda(x), axis, 128, INT8, signs=_cuda(s), rand_bits=_cuda(rb))
+    torch.cuda.synchronize()
+    along = 1 if axis == COLS else 0
+    v = oracle.rotate_signed(x, 128, along, s.numpy()[:n])
+    codes, scales, t = oracle.quantize_stochastic(v, 0 if along == 1 else 1, INT8, rb.numpy().view(np.uint16))
+    check_codes_stochastic(q, sc, codes, scales, t, rb.numpy().view(np.uint16), INT8)
+
+
+@pytest.mark.parametrize("blk", [128, 256])
+def test_linear_fwd_padded_k(blk):
+    m, n, k = 200, 136, 1000
+    x = inputs.activations(m, k, seed=61, device="cpu")
+    w = inputs.weights(n, k, seed=62, device="cpu")
+    y = halo.halo_linear_fwd(_cuda(x), _cuda(w), blk, INT8, FP32)
+    torch.cuda.synchronize()
+    check_output(y, oracle.linear_fwd(x, w, blk, INT8))
+
+
+def test_linear_bwd_padded_n_and_m():
+    m, n, k = 1000, 200, 256
+    dy = inputs.grads(m, n, seed=63, device="cpu")
+    x = inputs.activations(m, k, seed=64, device="cpu")
+    w = inputs.weights(n, k, seed=65, device="cpu")
+    dx, _ = halo.halo_linear_bwd(_cuda(dy), None, _cuda(w), 128, INT8, FP32, FP32, want_dw=False)
+    torch.cuda.synchronize()
+    check_output(dx, oracle.linear_bwd_dx(dy, w, 128, INT8))          # N = 200, padded to 256
+    n2 = 208  # dW needs N % 16
+    dy2 = inputs.grads(m, n2, seed=66, device="cpu")
+    _, dw = halo.halo_linear_bwd(_cuda(dy2), _cuda(x), None, 128, E4M3, FP32, FP32, want_dx=False)
+    torch.cuda.synchronize()
+    check_output(dw, oracle.linear_bwd_dw(dy2, x, 128, E4M3))         # M = 1000, padded to 1024
 
 
 # ------------------------------------------------------------------- edge cases
