@@ -619,6 +619,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="halo", choices=["halo", "reference"])
     ap.add_argument("--qtype", default="int8", choices=["int8", "e4m3"])
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel from the host instead of replaying the captured step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama70b_layer_fwd_bwd", choices=sorted(WORKLOADS),
@@ -640,6 +642,8 @@ def main():
     config = {"workload": args.workload, "tokens": shapes.tokens, "hidden": shapes.hidden,
               "ffn": shapes.ffn, "kv": shapes.kv, "gemms": len(shapes.gemms) * len(kinds), "block": BLK,
               "qtype": args.qtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
+    if args.impl != "reference":
+        config["launch"] = "stream" if args.no_graph else "cuda_graph"
 
     if args.impl == "reference":
         if rank != 0:
@@ -683,17 +687,42 @@ def main():
     if st != halo.HALO_OK:
         raise RuntimeError(f"device error after warm-up at site {site:#x}")
 
-    # Timed region: K plain steps (no events between launches).
+    # The step's launches captured once as a CUDA graph (same kernels, same
+    # arguments); replaying it keeps the GPU fed through the stretches of
+    # short kernels that per-launch host work (ctypes, tensor-map encoding)
+    # cannot keep up with.  --no-graph launches every kernel from the host.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            step.run()
+        torch.cuda.synchronize()
+        for _ in range(max(args.warmup, 3)):
+            graph.replay()
+        torch.cuda.synchronize()
+
+    # Timed region: K steps (no events between launches).
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_step = len(step.plan())
     with ClockSampler(local) as clocks:
         start.record(stream)
         launches = 0
         for _ in range(args.steps):
-            launches += step.run()
+            if graph is not None:
+                graph.replay()
+                launches += per_step
+            else:
+                launches += step.run()
         end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
