@@ -58,6 +58,8 @@ def _load():
         "halo_oracle_e4m3_encode": (ctypes.c_uint8, [D]),
         "halo_oracle_boundary_distance": (D, [D, I]),
         "halo_oracle_e4m3_encode_array": (None, [P, I64, P]),
+        "halo_oracle_quantize_grouped": (None, [P, I64, I64, I, I64, I, P, P, P]),
+        "halo_oracle_gemm_grouped": (None, [P, P, P, P, I64, I64, I64, I64, I, P]),
         "halo_oracle_e4m3_decode_array": (None, [P, I64, P]),
         "halo_oracle_boundary_distance_array": (None, [P, I64, I, P]),
         "halo_oracle_quantize": (None, [P, I64, I64, I, I, P, P, P]),
@@ -214,6 +216,71 @@ def quantize(v: np.ndarray, axis: int, qtype: int):
     t = np.empty((rows, cols), dtype=np.float64)
     _load().halo_oracle_quantize(_ptr(v), rows, cols, axis, qtype, _ptr(codes), _ptr(scales), _ptr(t))
     return codes, scales, t
+
+
+def quantize_grouped(v: np.ndarray, along: int, group: int, qtype: int):
+    """Group-wise scales along the contraction dimension: along=1 groups of
+    ``group`` consecutive elements of a row (scales [rows, cols/group]);
+    along=0 groups of ``group`` consecutive rows of a column (scales
+    [rows/group, cols]).  Returns (codes, scales, t)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, cols = v.shape
+    assert (cols if along == 1 else rows) % group == 0
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    shape = (rows, cols // group) if along == 1 else (rows // group, cols)
+    scales = np.empty(shape, dtype=np.float32)
+    t = np.empty((rows, cols), dtype=np.float64)
+    _load().halo_oracle_quantize_grouped(_ptr(v), rows, cols, along, group, qtype, _ptr(codes), _ptr(scales),
+                                         _ptr(t))
+    return codes, scales, t
+
+
+def gemm_grouped(a, sa, b, sb, group: int, qtype: int) -> np.ndarray:
+    """y[i, j] = sum_G sa[i, G] sb[j, G] sum_{k in G} a[i, k] b[j, k]; codes
+    [M, K] / [N, K] with the contraction dimension contiguous, scales [M, K/g] / [N, K/g]."""
+    a = np.ascontiguousarray(a).view(np.uint8)
+    b = np.ascontiguousarray(b).view(np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    m, k = a.shape
+    n, k2 = b.shape
+    assert k == k2 and k % group == 0 and sa.shape == (m, k // group) and sb.shape == (n, k // group)
+    y = np.empty((m, n), dtype=np.float64)
+    _load().halo_oracle_gemm_grouped(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), m, n, k, group, qtype, _ptr(y))
+    return y
+
+
+def grouped_operand(x, blk: int, along: int, group: int, qtype: int):
+    """Rotate (zero-padding as ``rotate``) and group-quantise one operand;
+    returns its codes and scales with the contraction dimension last:
+    ([outer, K], [outer, K/g]) whichever way the operand is stored."""
+    v = rotate(x, blk, along)
+    codes, scales, _ = quantize_grouped(v, along, group, qtype)
+    if along == 0:
+        codes, scales = codes.T, scales.T
+    return np.ascontiguousarray(codes), np.ascontiguousarray(scales)
+
+
+def linear_fwd_grouped(x, w, blk: int, group: int, qtype: int) -> np.ndarray:
+    """Y = X W^T with both operands rotated along K and quantised with one
+    scale per group of ``group`` consecutive K positions."""
+    xa, sx = grouped_operand(x, blk, 1, group, qtype)
+    wa, sw = grouped_operand(w, blk, 1, group, qtype)
+    return gemm_grouped(xa, sx, wa, sw, group, qtype)
+
+
+def linear_bwd_dx_grouped(dy, w, blk: int, group: int, qtype: int) -> np.ndarray:
+    """dX = dY W: dY rotated along N (its rows), W along N (dimension 0), group-wise along N."""
+    a, sa = grouped_operand(dy, blk, 1, group, qtype)
+    b, sb = grouped_operand(w, blk, 0, group, qtype)
+    return gemm_grouped(a, sa, b, sb, group, qtype)
+
+
+def linear_bwd_dw_grouped(dy, x, blk: int, group: int, qtype: int) -> np.ndarray:
+    """dW = dY^T X: both rotated along M (dimension 0), group-wise along M."""
+    a, sa = grouped_operand(dy, blk, 0, group, qtype)
+    b, sb = grouped_operand(x, blk, 0, group, qtype)
+    return gemm_grouped(a, sa, b, sb, group, qtype)
 
 
 def e4m3_encode(t) -> np.ndarray:

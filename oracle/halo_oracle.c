@@ -444,6 +444,86 @@ void halo_oracle_linear_bwd_dw(const uint16_t* dy, const uint16_t* x, int64_t m,
   halo_oracle_rotated_qgemm(dy, n, 0, x, k, 0, n, k, m, blk, qtype, dw, NULL, NULL);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Group-wise scales (QWHA page sec. 3.1, the quantiser's group_quantize:    */
+/* the values are cut into groups of group_size consecutive elements, each   */
+/* group with its own scale max|x| / qmax; sec. 3.2 recommends 64 and sec. 6 */
+/* 32-128).  Here a group runs along the GEMM's contraction dimension:       */
+/*   along = 1: `group` consecutive elements of a row; scales[rows][cols/g]  */
+/*   along = 0: `group` consecutive rows of a column;  scales[rows/g][cols]  */
+/* Within a group: s = (float)(amax / qmax) and the element rule of          */
+/* halo_oracle_quantize (round half to even and clamp to +-127, or E4M3).    */
+/* rows (along 0) or cols (along 1) must be a multiple of group.             */
+/* ------------------------------------------------------------------------ */
+void halo_oracle_quantize_grouped(const double* v, int64_t rows, int64_t cols, int along, int64_t group,
+                                  int qtype, uint8_t* codes, float* scales, double* t_out) {
+  const double qmax = (qtype == 0) ? 127.0 : 448.0;
+  const int64_t outer = (along == 1) ? rows : cols;          /* rows (along 1) or columns (along 0) */
+  const int64_t ngroups = ((along == 1) ? cols : rows) / group;
+  fesetround(FE_TONEAREST);
+  for (int64_t o = 0; o < outer; ++o) {
+    for (int64_t g = 0; g < ngroups; ++g) {
+      double amax = 0.0;
+      for (int64_t e = 0; e < group; ++e) {
+        int64_t idx = (along == 1) ? o * cols + g * group + e : (g * group + e) * cols + o;
+        double a = fabs(v[idx]);
+        if (a > amax) amax = a;
+      }
+      float s = (float)(amax / qmax);
+      if (along == 1)
+        scales[o * ngroups + g] = s;
+      else
+        scales[g * cols + o] = s;
+      for (int64_t e = 0; e < group; ++e) {
+        int64_t idx = (along == 1) ? o * cols + g * group + e : (g * group + e) * cols + o;
+        double t = (s == 0.0f) ? 0.0 : v[idx] / (double)s;
+        if (t_out) t_out[idx] = t;
+        if (qtype == 0) {
+          double q = nearbyint(t);
+          if (q > 127.0) q = 127.0;
+          if (q < -127.0) q = -127.0;
+          codes[idx] = (uint8_t)(int8_t)q;
+        } else {
+          codes[idx] = halo_oracle_e4m3_encode(t);
+        }
+      }
+    }
+  }
+}
+
+/* Product of group-quantised operands, both with the contraction dimension  */
+/* contiguous: A codes [M, K] with scales sa[M][K/g], B codes [N, K] with    */
+/* scales sb[N][K/g]:                                                        */
+/*   y[i, j] = sum_G sa[i][G] * sb[j][G] * sum_{k in group G} a[i, k] b[j, k] */
+/* Each group's sum is exact (int64 for INT8 codes, fp64 of the decoded E4M3 */
+/* values); the rest in fp64.                                                */
+void halo_oracle_gemm_grouped(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb, int64_t m,
+                              int64_t n, int64_t k, int64_t group, int qtype, double* y) {
+  const int64_t ng = k / group;
+  double lut[256];
+  for (int i = 0; i < 256; ++i) lut[i] = halo_oracle_e4m3_decode((uint8_t)i);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < m; ++i) {
+    for (int64_t j = 0; j < n; ++j) {
+      double sum = 0.0;
+      for (int64_t g = 0; g < ng; ++g) {
+        double part;
+        if (qtype == 0) {
+          int64_t acc = 0;
+          for (int64_t p = g * group; p < (g + 1) * group; ++p)
+            acc += (int64_t)(int8_t)a[i * k + p] * (int64_t)(int8_t)b[j * k + p];
+          part = (double)acc;
+        } else {
+          part = 0.0;
+          for (int64_t p = g * group; p < (g + 1) * group; ++p) part += lut[a[i * k + p]] * lut[b[j * k + p]];
+        }
+        sum += part * (double)sa[i * ng + g] * (double)sb[j * ng + g];
+      }
+      y[i * n + j] = sum;
+    }
+  }
+}
+
 int halo_oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

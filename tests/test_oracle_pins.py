@@ -518,3 +518,115 @@ def test_padding_is_zero_not_garbage():
     bad_w[:, 200:] = _bf16_bits(torch.ones(6, 56, dtype=torch.bfloat16))
     bad = oracle.rotate(bad_x, 128, 1) @ oracle.rotate(bad_w, 128, 1).T
     np.testing.assert_allclose(bad - exact, 56.0, rtol=1e-9)
+
+
+# ------------------------------------------------------------ group-wise scales
+def test_golden_grouped_quantisation():
+    for qt, group, inp, scales, codes in _rows("quantize_grouped_worked.txt"):
+        qtype = oracle.INT8 if qt == "int8" else oracle.E4M3
+        v = np.array([[float(t) for t in inp.split()]])
+        g = int(group)
+        q, s, _ = oracle.quantize_grouped(v, 1, g, qtype)
+        np.testing.assert_array_equal(s[0], np.array([float(x) for x in scales.split()], dtype=np.float32))
+        if qtype == oracle.INT8:
+            np.testing.assert_array_equal(q.view(np.int8)[0], [int(c) for c in codes.split()])
+        else:
+            np.testing.assert_array_equal(q[0], [int(c, 16) for c in codes.split()])
+        # the same values down a column (groups of consecutive rows)
+        qc, sc, _ = oracle.quantize_grouped(v.T.copy(), 0, g, qtype)
+        np.testing.assert_array_equal(qc[:, 0], q[0])
+        np.testing.assert_array_equal(sc[:, 0], s[0])
+
+
+@pytest.mark.parametrize("qtype", [oracle.INT8, oracle.E4M3])
+def test_grouped_with_one_group_is_the_per_row_quantiser(qtype):
+    rng = np.random.default_rng(41)
+    v = rng.standard_normal((7, 256)) * np.exp(rng.standard_normal((7, 1)))
+    q1, s1, t1 = oracle.quantize(v, 0, qtype)
+    qg, sg, tg = oracle.quantize_grouped(v, 1, 256, qtype)
+    np.testing.assert_array_equal(qg, q1)
+    np.testing.assert_array_equal(sg[:, 0], s1)
+    np.testing.assert_array_equal(tg, t1)
+    qc, sc, _ = oracle.quantize_grouped(v.T.copy(), 0, 256, qtype)     # one group down each column
+    q0, s0, _ = oracle.quantize(v.T.copy(), 1, qtype)
+    np.testing.assert_array_equal(qc, q0)
+    np.testing.assert_array_equal(sc[0], s0)
+
+
+def test_grouped_int8_bounds():
+    rng = np.random.default_rng(42)
+    v = rng.standard_normal((9, 512))
+    v[2, 100] = 77.0
+    q, s, _ = oracle.quantize_grouped(v, 1, 64, oracle.INT8)
+    qi = q.view(np.int8).astype(np.int64).reshape(9, 8, 64)
+    vg = v.reshape(9, 8, 64)
+    assert np.all(np.abs(qi) <= 127)
+    assert np.all(np.abs(qi).max(axis=2) == 127)             # every group's max maps to +-qmax
+    sd = s.astype(np.float64)[:, :, None]
+    assert np.all(np.abs(vg - qi * sd) <= sd / 2 * (1 + 1e-6))
+    # an outlier only coarsens its own group
+    assert s[2, 1] > 20 * np.median(s)
+    assert np.sum(s > 20 * np.median(s)) == 1
+
+
+def test_grouped_gemm_against_numpy_group_sums():
+    """numpy computes each group's integer product on its own (einsum over the
+    group axis) and weights it by the two scales: a swapped or transposed
+    group index anywhere in the oracle fails this."""
+    rng = np.random.default_rng(43)
+    m, n, k, g = 12, 10, 256, 64
+    a = rng.integers(-127, 128, (m, k)).astype(np.int8)
+    b = rng.integers(-127, 128, (n, k)).astype(np.int8)
+    sa = rng.uniform(0.5, 2.0, (m, k // g)).astype(np.float32)
+    sb = rng.uniform(0.5, 2.0, (n, k // g)).astype(np.float32)
+    y = oracle.gemm_grouped(a.view(np.uint8), sa, b.view(np.uint8), sb, g, oracle.INT8)
+    parts = np.einsum("igk,jgk->ijg", a.reshape(m, k // g, g).astype(np.int64), b.reshape(n, k // g, g).astype(np.int64))
+    expect = np.einsum("ijg,ig,jg->ij", parts.astype(np.float64), sa.astype(np.float64), sb.astype(np.float64))
+    np.testing.assert_allclose(y, expect, rtol=1e-12)
+    # unit scales: the plain integer product
+    ones_a, ones_b = np.ones((m, k // g), np.float32), np.ones((n, k // g), np.float32)
+    np.testing.assert_array_equal(oracle.gemm_grouped(a.view(np.uint8), ones_a, b.view(np.uint8), ones_b, g,
+                                                      oracle.INT8), (a.astype(np.int64) @ b.astype(np.int64).T))
+    # E4M3 on torch-decoded values
+    ca = rng.integers(0, 256, (m, k)).astype(np.uint8)
+    cb = rng.integers(0, 256, (n, k)).astype(np.uint8)
+    ca[(ca & 0x7F) == 0x7F] = 0   # no NaN codes
+    cb[(cb & 0x7F) == 0x7F] = 0
+    da = torch.from_numpy(ca).view(torch.float8_e4m3fn).double().numpy().reshape(m, k // g, g)
+    db = torch.from_numpy(cb).view(torch.float8_e4m3fn).double().numpy().reshape(n, k // g, g)
+    expect = np.einsum("igk,jgk,ig,jg->ij", da, db, sa.astype(np.float64), sb.astype(np.float64))
+    np.testing.assert_allclose(oracle.gemm_grouped(ca, sa, cb, sb, g, oracle.E4M3), expect, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_linear_layers_within_quantisation_bound():
+    """The three products with group-wise scales (g = 64) stay within the
+    worst-case bound of their per-group quantisation errors around the exact
+    products, and are tighter than the per-row scales on outlier inputs."""
+    rng = np.random.default_rng(44)
+    m, n, k, blk, g = 256, 128, 384, 128, 64
+    xf = torch.from_numpy(rng.standard_normal((m, k)).astype(np.float32))
+    xf[:, 9] *= 50
+    x = xf.to(torch.bfloat16)
+    w = torch.from_numpy((0.02 * rng.standard_normal((n, k))).astype(np.float32)).to(torch.bfloat16)
+    dy = torch.from_numpy((1e-3 * rng.standard_normal((m, n))).astype(np.float32)).to(torch.bfloat16)
+    xd, wd, dyd = x.double().numpy(), w.double().numpy(), dy.double().numpy()
+
+    def bound(a_rot, b_rot, along_a, along_b):
+        # per-element INT8 errors <= s/2 of the element's own group
+        def err(v, along):
+            _, s, _ = oracle.quantize_grouped(v, along, g, oracle.INT8)
+            e = np.repeat(0.5 * s.astype(np.float64), g, axis=1 if along == 1 else 0)
+            return (e if along == 1 else e.T), (v if along == 1 else v.T)
+        ea, va = err(a_rot, along_a)
+        eb, vb = err(b_rot, along_b)
+        return ea @ np.abs(vb).T + np.abs(va) @ eb.T + ea @ eb.T
+
+    y = oracle.linear_fwd_grouped(x, w, blk, g, oracle.INT8)
+    exact = xd @ wd.T
+    assert np.all(np.abs(y - exact) <= bound(oracle.rotate(x, blk, 1), oracle.rotate(w, blk, 1), 1, 1) * (1 + 1e-9) + 1e-15)
+    yr = oracle.linear_fwd(x, w, blk, oracle.INT8)
+    assert np.abs(y - exact).max() < np.abs(yr - exact).max()
+    dx = oracle.linear_bwd_dx_grouped(dy, w, blk, g, oracle.INT8)
+    assert np.all(np.abs(dx - dyd @ wd) <= bound(oracle.rotate(dy, blk, 1), oracle.rotate(w, blk, 0), 1, 0) * (1 + 1e-9) + 1e-15)
+    dw = oracle.linear_bwd_dw_grouped(dy, x, blk, g, oracle.INT8)
+    assert np.all(np.abs(dw - dyd.T @ xd) <= bound(oracle.rotate(dy, blk, 0), oracle.rotate(x, blk, 0), 0, 0) * (1 + 1e-9) + 1e-15)
