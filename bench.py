@@ -113,10 +113,12 @@ class ClockSampler:
 class LayerStep:
     """All tensors and launches of one layer step (forward + dX + dW of 7 GEMMs)."""
 
-    def __init__(self, shapes: inputs.LayerShapes, seed: int, device, qtype: int, kinds=("fwd", "dx", "dw")):
+    def __init__(self, shapes: inputs.LayerShapes, seed: int, device, qtype: int, kinds=("fwd", "dx", "dw"),
+                 group: int = 0):
         import hadamard_rotated_precision_halo_b200 as halo
 
         self.halo = halo
+        self.group = group  # 0: one scale per row / column; 64 or 128: group-wise scales along K
         self.kinds = kinds
         self.shapes = shapes
         self.qtype = qtype
@@ -132,15 +134,20 @@ class LayerStep:
         # Code / scale buffers for the two operands of the GEMM in flight.
         self.qa = torch.empty(max(max_mk, max_mn), dtype=torch.uint8, device=device)
         self.qb = torch.empty(max(max_nk, max_mk), dtype=torch.uint8, device=device)
-        self.sa = torch.empty(max_vec, dtype=torch.float32, device=device)
-        self.sb = torch.empty(max_vec, dtype=torch.float32, device=device)
+        n_scales = max(max_vec, max(max_mk, max_nk, max_mn) // group) if group else max_vec
+        self.sa = torch.empty(n_scales, dtype=torch.float32, device=device)
+        self.sb = torch.empty(n_scales, dtype=torch.float32, device=device)
         self.code_dt = code_dt
         for g in shapes.gemms:
             self.y[g.name] = torch.empty((t, g.n), dtype=torch.bfloat16, device=device)
             self.dx[g.name] = torch.empty((t, g.k), dtype=torch.bfloat16, device=device)
             self.dw[g.name] = torch.empty((g.n, g.k), dtype=torch.float32, device=device)
-        self.ws_fwd = max(halo.halo_workspace_size(t, g.n, g.k, 0) for g in shapes.gemms)
-        self.ws_bwd = max(halo.halo_workspace_size(t, g.n, g.k, 1) for g in shapes.gemms)
+        if group:
+            wsz = lambda m, n, k, which: int(halo.lib().halo_workspace_size_grouped(m, n, k, group, which))
+        else:
+            wsz = halo.halo_workspace_size
+        self.ws_fwd = max(wsz(t, g.n, g.k, 0) for g in shapes.gemms)
+        self.ws_bwd = max(wsz(t, g.n, g.k, 1) for g in shapes.gemms)
         self.ws = torch.empty(max(self.ws_fwd, self.ws_bwd), dtype=torch.uint8, device=device)
 
     def ops_per_step(self) -> int:
@@ -148,6 +155,14 @@ class LayerStep:
 
     def _codes(self, buf, rows, cols):
         return buf[: rows * cols].view(self.code_dt).view(rows, cols)
+
+    def n_scales(self, x, ax) -> int:
+        """Scales of one rotate+quantise of x along axis ax: one per row / column,
+        or one per group of the rotated dimension."""
+        rows, cols = x.shape
+        if ax == self.halo.HALO_AXIS_COLS:
+            return rows * (cols // self.group if self.group else 1)
+        return cols * (rows // self.group if self.group else 1)
 
     def gemms(self):
         """The step as (a, a_axis, b, b_axis, m, n, k, out) launch groups, in order."""
@@ -187,9 +202,8 @@ class LayerStep:
             for x, ax in ((g[2], g[3]), (g[4], g[5])):
                 key = (x.data_ptr(), ax)
                 if count[key] > 1 and key not in self.shared:
-                    groups = x.shape[0] if ax == h.HALO_AXIS_COLS else x.shape[1]
                     q = torch.empty(x.shape, dtype=self.code_dt, device=self.dev)
-                    sc = torch.empty(groups, dtype=torch.float32, device=self.dev)
+                    sc = torch.empty(self.n_scales(x, ax), dtype=torch.float32, device=self.dev)
                     self.shared[key] = (q, sc)
         plan, done = [], set()
         for kind, name, a, a_axis, b, b_axis, m, n, k, c in gem:
@@ -226,16 +240,26 @@ class LayerStep:
                 events.append(ev)
             if op[0] == "rotq":
                 _, x, ax, q, sc = op
-                st = L.halo_hadamard_quantize(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), ax, BLK, self.qtype,
-                                              h._ptr(q), q.stride(0), h._ptr(sc), sp)
+                if self.group:
+                    st = L.halo_hadamard_quantize_grouped(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), ax, BLK,
+                                                          self.group, self.qtype, h._ptr(q), q.stride(0), h._ptr(sc),
+                                                          sp)
+                else:
+                    st = L.halo_hadamard_quantize(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), ax, BLK,
+                                                  self.qtype, h._ptr(q), q.stride(0), h._ptr(sc), sp)
                 h._check(st, "halo_hadamard_quantize")
             else:
                 _, (qa, sa, ax_a), (qb, sb, ax_b), m, n, k, c = op
                 a_major = h.HALO_MAJOR_K if ax_a == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
                 b_major = h.HALO_MAJOR_K if ax_b == h.HALO_AXIS_COLS else h.HALO_MAJOR_MN
                 otype = h.HALO_OUT_FP32 if c.dtype == torch.float32 else h.HALO_OUT_BF16
-                st = L.halo_qgemm(h._ptr(qa), h._ptr(sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(sb), b_major,
-                                  qb.stride(0), m, n, k, self.qtype, h._ptr(c), otype, c.stride(0), sp)
+                if self.group:
+                    st = L.halo_qgemm_grouped(h._ptr(qa), h._ptr(sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(sb),
+                                              b_major, qb.stride(0), m, n, k, self.group, self.qtype, h._ptr(c),
+                                              otype, c.stride(0), sp)
+                else:
+                    st = L.halo_qgemm(h._ptr(qa), h._ptr(sa), a_major, qa.stride(0), h._ptr(qb), h._ptr(sb),
+                                      b_major, qb.stride(0), m, n, k, self.qtype, h._ptr(c), otype, c.stride(0), sp)
                 h._check(st, "halo_qgemm")
         if events is not None:
             ev = torch.cuda.Event(enable_timing=True)
@@ -268,8 +292,7 @@ class LayerStep:
         for op in self.plan():
             if op[0] == "rotq":
                 x, ax = op[1], op[2]
-                groups = x.shape[0] if ax == h.HALO_AXIS_COLS else x.shape[1]
-                total += 3 * x.numel() + 4 * groups
+                total += 3 * x.numel() + 4 * self.n_scales(x, ax)
         return total
 
     def gemm_bytes(self) -> int:
@@ -279,7 +302,8 @@ class LayerStep:
         for op in self.plan():
             if op[0] == "gemm":
                 m, n, k, c = op[3], op[4], op[5], op[6]
-                total += m * k + n * k + m * n * c.element_size() + 4 * (m + n)
+                ng = k // self.group if self.group else 1
+                total += m * k + n * k + m * n * c.element_size() + 4 * (m + n) * ng
         return total
 
     def gemm_ops(self) -> int:
@@ -341,14 +365,23 @@ def e2e_run(step: LayerStep, steps: int):
         for g in gemms:
             comp.wait_event(ready[("x", g.x_key)])
             comp.wait_event(ready[("w", g.name)])
-            h.halo_linear_fwd(din["x"][g.x_key], din["w"][g.name], BLK, step.qtype, h.HALO_OUT_BF16,
-                              y=dout["y"][g.name], ws=step.ws, stream=comp)
+            if step.group:
+                h.halo_linear_fwd_grouped(din["x"][g.x_key], din["w"][g.name], BLK, step.group, step.qtype,
+                                          h.HALO_OUT_BF16, y=dout["y"][g.name], ws=step.ws, stream=comp)
+            else:
+                h.halo_linear_fwd(din["x"][g.x_key], din["w"][g.name], BLK, step.qtype, h.HALO_OUT_BF16,
+                                  y=dout["y"][g.name], ws=step.ws, stream=comp)
             done.append((("y", g.name), event(comp)))
         for g in gemms:
             comp.wait_event(ready[("dy", g.name)])
-            h.halo_linear_bwd(din["dy"][g.name], din["x"][g.x_key], din["w"][g.name], BLK, step.qtype,
-                              h.HALO_OUT_BF16, h.HALO_OUT_FP32, dx=dout["dx"][g.name], dw=dout["dw"][g.name],
-                              ws=step.ws, stream=comp)
+            if step.group:
+                h.halo_linear_bwd_grouped(din["dy"][g.name], din["x"][g.x_key], din["w"][g.name], BLK, step.group,
+                                          step.qtype, h.HALO_OUT_BF16, h.HALO_OUT_FP32, dx=dout["dx"][g.name],
+                                          dw=dout["dw"][g.name], ws=step.ws, stream=comp)
+            else:
+                h.halo_linear_bwd(din["dy"][g.name], din["x"][g.x_key], din["w"][g.name], BLK, step.qtype,
+                                  h.HALO_OUT_BF16, h.HALO_OUT_FP32, dx=dout["dx"][g.name], dw=dout["dw"][g.name],
+                                  ws=step.ws, stream=comp)
             e = event(comp)
             done += [(("dx", g.name), e), (("dw", g.name), e)]
         inputs_free[b] = event(comp)
@@ -554,6 +587,30 @@ def measure_rotq_shapes(repeats: int = 10):
         out.append({"direction": "along_contiguous_dim", "shape": [r, c], "qtype": "int8+e4m3 (one read)",
                     "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
         del x, outs
+    # Group-wise scales (halo_hadamard_quantize_grouped, INT8): 4 B per scale
+    # of every group of 64 / 128 positions along the rotated dimension.
+    for name, shapes in ROTQ_SHAPES.items():
+        axis = halo.HALO_AXIS_COLS if name == "along_contiguous_dim" else halo.HALO_AXIS_ROWS
+        for r, c in (shapes[1], shapes[-1]):
+            x = inputs.activations(r, c, seed=1, device="cuda")
+            for group in (64, 128):
+                q, sc = halo.halo_hadamard_quantize_grouped(x, axis, BLK, group, halo.HALO_Q_INT8)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(repeats):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    halo.halo_hadamard_quantize_grouped(x, axis, BLK, group, halo.HALO_Q_INT8, q_out=q, scales_out=sc)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                ms = sorted(ts)[len(ts) // 2]
+                nbytes = 3 * x.numel() + 4 * sc.numel()
+                out.append({"direction": name, "shape": [r, c], "qtype": "int8", "variant": f"group {group}",
+                            "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
+                del q, sc
+            del x
     # The variants (halo_hadamard_quantize_ex): random signs along the rotated
     # dimension and stochastic rounding from 16 random bits per element (which
     # add 2 B per element of input traffic).
@@ -619,6 +676,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="halo", choices=["halo", "reference"])
     ap.add_argument("--qtype", default="int8", choices=["int8", "e4m3"])
+    ap.add_argument("--group", type=int, default=0, choices=[0, 64, 128],
+                    help="group-wise scales along each GEMM's contraction dimension (0: one scale per row)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying the captured step")
     ap.add_argument("--no-e2e", action="store_true")
@@ -644,6 +703,8 @@ def main():
               "qtype": args.qtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
     if args.impl != "reference":
         config["launch"] = "stream" if args.no_graph else "cuda_graph"
+        if args.group:
+            config["scale_group"] = args.group
 
     if args.impl == "reference":
         if rank != 0:
@@ -677,7 +738,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     qtype = halo.HALO_Q_INT8 if args.qtype == "int8" else halo.HALO_Q_E4M3
-    step = LayerStep(shapes, seed=4 + rank, device=device, qtype=qtype, kinds=kinds)
+    step = LayerStep(shapes, seed=4 + rank, device=device, qtype=qtype, kinds=kinds, group=args.group)
     torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
@@ -761,10 +822,11 @@ def main():
             "vs_baseline": None, "dtype": "int8" if qtype == halo.HALO_Q_INT8 else "e4m3",
             "data": "synthetic", "config": config,
             "gpu_launches": launches,
-            "roofline": {"bound": "tensor", "kernel": "qgemm_pair_kernel", "achieved": gemm_tops, "peak": peak8,
-                         "unit": "TFLOP/s", "frac": gemm_tops / peak8,
+            "roofline": {"bound": "tensor", "kernel": "qgemm_grouped_kernel" if args.group else "qgemm_pair_kernel",
+                         "achieved": gemm_tops, "peak": peak8, "unit": "TFLOP/s", "frac": gemm_tops / peak8,
                          "traffic": (GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER
-                                     if args.workload == "llama70b_layer_fwd_bwd" and args.qtype == "int8" else None),
+                                     if args.workload == "llama70b_layer_fwd_bwd" and args.qtype == "int8"
+                                     and not args.group else None),
                          "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                          "algorithmic_bytes_per_launch": step.gemm_bytes() / max(n_gemm // args.steps, 1),
                          "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']}); "

@@ -41,6 +41,11 @@ EXPORTS = (
     "halo_hadamard_quantize",
     "halo_hadamard_quantize_ex",
     "halo_hadamard_quantize_dual",
+    "halo_hadamard_quantize_grouped",
+    "halo_qgemm_grouped",
+    "halo_workspace_size_grouped",
+    "halo_linear_fwd_grouped",
+    "halo_linear_bwd_grouped",
     "halo_qgemm",
     "halo_workspace_size",
     "halo_linear_fwd",
@@ -82,6 +87,16 @@ def lib():
     L.halo_hadamard_quantize_ex.restype = I
     L.halo_hadamard_quantize_dual.argtypes = [P, I64, I64, I64, I, P, I64, P, P, I64, P, P]
     L.halo_hadamard_quantize_dual.restype = I
+    L.halo_hadamard_quantize_grouped.argtypes = [P, I64, I64, I64, I, I, I, I, P, I64, P, P]
+    L.halo_hadamard_quantize_grouped.restype = I
+    L.halo_qgemm_grouped.argtypes = [P, P, I, I64, P, P, I, I64, I64, I64, I64, I, I, P, I, I64, P]
+    L.halo_qgemm_grouped.restype = I
+    L.halo_workspace_size_grouped.argtypes = [I64, I64, I64, I, I]
+    L.halo_workspace_size_grouped.restype = SZ
+    L.halo_linear_fwd_grouped.argtypes = [P, P, I64, I64, I64, I, I, I, P, I, P, SZ, P]
+    L.halo_linear_fwd_grouped.restype = I
+    L.halo_linear_bwd_grouped.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I, P, I, P, SZ, P]
+    L.halo_linear_bwd_grouped.restype = I
     L.halo_qgemm.argtypes = [P, P, I, I64, P, P, I, I64, I64, I64, I64, I, P, I, I64, P]
     L.halo_qgemm.restype = I
     L.halo_workspace_size.argtypes = [I64, I64, I64, I]
@@ -200,6 +215,65 @@ def halo_hadamard_quantize_dual(x: torch.Tensor, blk: int, q_int8=None, scales_i
                                            _stream(stream))
     _check(st, "halo_hadamard_quantize_dual")
     return q_int8, scales_int8, q_e4m3, scales_e4m3
+
+
+def halo_hadamard_quantize_grouped(x: torch.Tensor, axis: int, blk: int, group: int, qtype: int, q_out=None,
+                                   scales_out=None, stream=None):
+    """Rotate + quantise with one scale per `group` positions along the rotated
+    dimension; returns (codes, scales) with scales [rows, cols_p/group]
+    (HALO_AXIS_COLS) or [rows_p/group, cols] (HALO_AXIS_ROWS)."""
+    rows, cols = x.shape
+    shape = codes_shape(rows, cols, axis, blk)
+    if q_out is None:
+        q_out = torch.empty(shape, dtype=_code_dtype(qtype), device=x.device)
+    if scales_out is None:
+        sshape = (rows, shape[1] // group) if axis == HALO_AXIS_COLS else (shape[0] // group, cols)
+        scales_out = torch.empty(sshape, dtype=torch.float32, device=x.device)
+    st = lib().halo_hadamard_quantize_grouped(_ptr(x), rows, cols, x.stride(0), axis, blk, group, qtype, _ptr(q_out),
+                                              q_out.stride(0), _ptr(scales_out), _stream(stream))
+    _check(st, "halo_hadamard_quantize_grouped")
+    return q_out, scales_out
+
+
+def halo_qgemm_grouped(a_q, s_a, a_major, b_q, s_b, b_major, m, n, k, group, qtype, otype, c=None, stream=None):
+    """C[m, n] = sum_G s_a[., G] s_b[., G] (A_G B_G^T) on 8-bit codes with group-wise scales."""
+    if c is None:
+        c = torch.empty((m, n), dtype=_out_dtype(otype), device=a_q.device)
+    st = lib().halo_qgemm_grouped(_ptr(a_q), _ptr(s_a), a_major, a_q.stride(0), _ptr(b_q), _ptr(s_b), b_major,
+                                  b_q.stride(0), m, n, k, group, qtype, _ptr(c), otype, c.stride(0), _stream(stream))
+    _check(st, "halo_qgemm_grouped")
+    return c
+
+
+def halo_linear_fwd_grouped(x, w, blk, group, qtype, otype, y=None, ws=None, stream=None):
+    m, k = x.shape
+    n = w.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=_out_dtype(otype), device=x.device)
+    if ws is None:
+        ws = torch.empty(int(lib().halo_workspace_size_grouped(m, n, k, group, 0)), dtype=torch.uint8, device=x.device)
+    st = lib().halo_linear_fwd_grouped(_ptr(x), _ptr(w), m, n, k, blk, group, qtype, _ptr(y), otype, _ptr(ws),
+                                       ws.numel(), _stream(stream))
+    _check(st, "halo_linear_fwd_grouped")
+    return y
+
+
+def halo_linear_bwd_grouped(dy, x, w, blk, group, qtype, otype_dx, otype_dw, dx=None, dw=None, want_dx=True,
+                            want_dw=True, ws=None, stream=None):
+    m, n = dy.shape
+    k = (x if x is not None else w).shape[1]
+    dev = dy.device
+    if want_dx and dx is None:
+        dx = torch.empty((m, k), dtype=_out_dtype(otype_dx), device=dev)
+    if want_dw and dw is None:
+        dw = torch.empty((n, k), dtype=_out_dtype(otype_dw), device=dev)
+    if ws is None:
+        ws = torch.empty(int(lib().halo_workspace_size_grouped(m, n, k, group, 1)), dtype=torch.uint8, device=dev)
+    st = lib().halo_linear_bwd_grouped(_ptr(dy), _ptr(x), _ptr(w), m, n, k, blk, group, qtype,
+                                       _ptr(dx if want_dx else None), otype_dx, _ptr(dw if want_dw else None),
+                                       otype_dw, _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "halo_linear_bwd_grouped")
+    return dx, dw
 
 
 def halo_qgemm(a_q, s_a, a_major, b_q, s_b, b_major, m, n, k, qtype, otype, c=None, stream=None):

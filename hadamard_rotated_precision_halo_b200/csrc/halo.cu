@@ -12,6 +12,7 @@
 
 #include "../../include/halo.h"
 #include "qgemm.cuh"
+#include "qgemm_grouped.cuh"
 #include "rotq.cuh"
 
 using namespace halo;
@@ -73,6 +74,12 @@ typedef void (*Cols2Kernel)(const CUtensorMap, const CUtensorMap, RotqColsParams
 // `ext`: the instantiation that reads the variants' optional inputs (signs,
 // random bits); the plain path is compiled without them.
 template <int PAD>
+RowsKernel rows_kernel_grouped_for(int blk, int qtype) {
+  if (blk == 128) return qtype == HALO_Q_INT8 ? rotq_rows_kernel<128, 0, 0, PAD, 1> : rotq_rows_kernel<128, 1, 0, PAD, 1>;
+  return qtype == HALO_Q_INT8 ? rotq_rows_kernel<256, 0, 0, PAD, 1> : rotq_rows_kernel<256, 1, 0, PAD, 1>;
+}
+
+template <int PAD>
 RowsKernel rows_kernel_for(int blk, int qtype, bool ext) {
   if (qtype == kQtDual)
     return blk == 128 ? rotq_rows_kernel<128, kQtDual, 0, PAD> : rotq_rows_kernel<256, kQtDual, 0, PAD>;
@@ -86,9 +93,13 @@ RowsKernel rows_kernel_for(int blk, int qtype, bool ext) {
 
 // qtype kQtDual (2): INT8 and E4M3 codes from one read (plain path only).
 // pad: the row length is not a multiple of the block.
-RowsKernel rows_kernel(int blk, int qtype, bool ext, bool pad) {
+// grouped: group-wise scales (qtype INT8 / E4M3, plain path only).
+RowsKernel rows_kernel(int blk, int qtype, bool ext, bool pad, bool grouped = false) {
+  if (grouped) return pad ? rows_kernel_grouped_for<1>(blk, qtype) : rows_kernel_grouped_for<0>(blk, qtype);
   return pad ? rows_kernel_for<1>(blk, qtype, ext) : rows_kernel_for<0>(blk, qtype, ext);
 }
+
+typedef void (*ColsGrKernel)(const CUtensorMap, const CUtensorMap, RotqColsGrParams);
 
 template <int QT, int EXT>
 Cols1Kernel cols_1pass_for(int nw) {
@@ -139,7 +150,15 @@ halo_status_t device_setup(int* dev_out) {
     }
     int optin = 0;
     HALO_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    HALO_CUDA(set_smem_attr(rotq_cols_grouped_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(rotq_cols_grouped_kernel<1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_grouped_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_grouped_kernel<1>, optin));
     for (int pad = 0; pad < 2; ++pad) {
+      for (int qt = 0; qt < 2; ++qt) {
+        HALO_CUDA(set_smem_attr(rows_kernel(128, qt, false, pad, true), optin));
+        HALO_CUDA(set_smem_attr(rows_kernel(256, qt, false, pad, true), optin));
+      }
       HALO_CUDA(set_smem_attr(rows_kernel(128, kQtDual, false, pad), optin));
       HALO_CUDA(set_smem_attr(rows_kernel(256, kQtDual, false, pad), optin));
       for (int e = 0; e < 2; ++e) {
@@ -238,7 +257,7 @@ int64_t pad_to(int64_t n, int64_t b) { return (n + b - 1) / b * b; }
 halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
                                void* q, int64_t ld_q, float* scales, const RotqExtras& ex, bool ext,
                                cudaStream_t stream, int dev, void* q2 = nullptr, int64_t ld_q2 = 0,
-                               float* scales2 = nullptr) {
+                               float* scales2 = nullptr, int group = 0) {
   const bool dual = qtype == kQtDual;
   // A row of `cols` elements is zero-padded to whole blocks: nb 128-element
   // chunks, of which nbt are whole in the input and one more (tail > 0
@@ -303,8 +322,9 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   p.ex = ex;
   p.scales2 = scales2;
   p.scale_mult2 = static_cast<float>(1.0 / (448.0 * sqrt(static_cast<double>(blk))));
+  p.group = group;
 
-  RowsKernel kern = rows_kernel(blk, qtype, ext, pad);
+  RowsKernel kern = rows_kernel(blk, qtype, ext, pad, group != 0);
   int per_sm = 0;
   HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
   if (per_sm < 1) per_sm = 1;
@@ -406,6 +426,109 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
 
   Launch L(dim3(cl, strips, 1), dim3(32 * warps), smem, stream, cl);
   HALO_CUDA(cudaLaunchKernelEx(&L.cfg, cols_2pass_kernel(qtype, ext), tm_x, tm_q, p));
+  return HALO_OK;
+}
+
+// Dimension-0 rotation with group-wise scales: independent warps over the
+// (128-row block, 32-column strip) items; scales [rows_p / group][cols].
+halo_status_t launch_rotq_cols_grouped(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
+                                       int64_t ld_q, float* scales, int group, cudaStream_t stream, int dev) {
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(pad_to(rows, 128))};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  RotqColsGrParams p;
+  p.scales = scales;
+  p.cols = cols;
+  p.strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
+  p.nblocks = static_cast<int>(pad_to(rows, 128) / 128);
+  p.group = group;
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  ColsGrKernel kern = qtype == HALO_Q_INT8 ? rotq_cols_grouped_kernel<0> : rotq_cols_grouped_kernel<1>;
+  const size_t smem = 4 * (2 * kColsInBytes) + 128;
+  int per_sm = 0;
+  HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, smem));
+  if (per_sm < 1) per_sm = 1;
+  const int64_t items = static_cast<int64_t>(p.nblocks) * p.strips;
+  const int grid = static_cast<int>(std::min<int64_t>((items + 3) / 4, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
+  Launch L(dim3(grid), dim3(128), smem, stream, 0);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
+// GEMM with group-wise scales: 128 x 128 tiles, one CTA per SM, persistent.
+// Scale of (row i, group G) of a K-major operand [outer, K]: s[i * K/g + G];
+// of an MN-major operand [K, outer]: s[G * outer + i].
+halo_status_t launch_qgemm_grouped(const void* a, const float* sa, int a_mn, int64_t ld_a, const void* b,
+                                   const float* sb, int b_mn, int64_t ld_b, int64_t m, int64_t n, int64_t k,
+                                   int group, int qtype, void* c, int otype, int64_t ld_c, cudaStream_t stream,
+                                   int dev) {
+  CUtensorMap tm_a, tm_b;
+  const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a_mn ? m : k), static_cast<cuuint64_t>(a_mn ? k : m)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_a)};
+    cuuint32_t box[2] = {128, 128};
+    halo_status_t st = encode(&tm_a, dt, 2, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(b_mn ? n : k), static_cast<cuuint64_t>(b_mn ? k : n)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_b)};
+    cuuint32_t box[2] = {128, 128};
+    halo_status_t st = encode(&tm_b, dt, 2, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != HALO_OK) return st;
+  }
+  GroupedGemmParams p;
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.group = group;
+  p.tiles_m = static_cast<int>((m + kGgBM - 1) / kGgBM);
+  p.tiles_n = static_cast<int>((n + kGgBN - 1) / kGgBN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
+  uint32_t idesc = 0;
+  if (qtype == HALO_Q_INT8)
+    idesc |= (2u << 4) | (1u << 7) | (1u << 10);  // s32 accumulate, signed 8-bit A and B
+  else
+    idesc |= (1u << 4);                           // f32 accumulate, E4M3 A and B
+  idesc |= static_cast<uint32_t>(a_mn) << 15;
+  idesc |= static_cast<uint32_t>(b_mn) << 16;
+  idesc |= static_cast<uint32_t>(kGgBN >> 3) << 17;
+  idesc |= static_cast<uint32_t>(kGgBM >> 4) << 24;
+  p.idesc = idesc;
+  const int64_t ng = k / group;
+  p.sa = sa;
+  p.sa_row = a_mn ? 1 : ng;
+  p.sa_grp = a_mn ? m : 1;
+  p.sb = sb;
+  p.sb_row = b_mn ? 1 : ng;
+  p.sb_grp = b_mn ? n : 1;
+  p.c = c;
+  p.ldc = ld_c;
+  p.out_bf16 = otype == HALO_OUT_BF16;
+  const int grid = std::min(p.num_tiles, g_dev[dev].sm_count);
+  Launch L(dim3(grid), dim3(kGgThreads), kGgSmemBytes, stream, 0);
+  if (qtype == HALO_Q_INT8)
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_grouped_kernel<0>, tm_a, tm_b, p));
+  else
+    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_grouped_kernel<1>, tm_a, tm_b, p));
   return HALO_OK;
 }
 
@@ -558,27 +681,30 @@ struct WsLayout {
 // Scratch of the linear layers: codes and scales of both operands of each GEMM,
 // the contraction dimension zero-padded to whole blocks (fwd: K to blk; dX: N
 // to 128; dW: M to 128).
-WsLayout ws_layout(int64_t m, int64_t n, int64_t k, int which, int blk) {
+// group > 0: group-wise scales, one per `group` positions of the contraction
+// dimension instead of one per operand row.
+WsLayout ws_layout(int64_t m, int64_t n, int64_t k, int which, int blk, int group = 0) {
   WsLayout L = {};
   size_t sizes[8];
   int cnt;
+  auto ngroups = [&](int64_t len) { return static_cast<size_t>(group ? len / group : 1); };
   if (which == 0) {
     const int64_t kp = pad_to(k, blk);
     sizes[0] = size_t(m) * kp;
     sizes[1] = size_t(n) * kp;
-    sizes[2] = size_t(m) * 4;
-    sizes[3] = size_t(n) * 4;
+    sizes[2] = size_t(m) * ngroups(kp) * 4;
+    sizes[3] = size_t(n) * ngroups(kp) * 4;
     cnt = 4;
   } else {
     const int64_t np = pad_to(n, 128), mp = pad_to(m, 128);
     sizes[0] = size_t(m) * np;
     sizes[1] = size_t(np) * k;
-    sizes[2] = size_t(m) * 4;
-    sizes[3] = size_t(k) * 4;
+    sizes[2] = size_t(m) * ngroups(np) * 4;
+    sizes[3] = size_t(k) * ngroups(np) * 4;
     sizes[4] = size_t(mp) * n;
     sizes[5] = size_t(mp) * k;
-    sizes[6] = size_t(n) * 4;
-    sizes[7] = size_t(k) * 4;
+    sizes[6] = size_t(n) * ngroups(mp) * 4;
+    sizes[7] = size_t(k) * ngroups(mp) * 4;
     cnt = 8;
   }
   size_t off = 0;
@@ -677,6 +803,46 @@ halo_status_t halo_hadamard_quantize_dual(const void* x_bf16, int64_t rows, int6
                           static_cast<cudaStream_t>(stream), dev, q_e4m3, ld_qf8, scales_e4m3);
 }
 
+halo_status_t halo_hadamard_quantize_grouped(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                                             int axis, int blk, int group, int qtype, void* q_out, int64_t ld_q,
+                                             float* scales_out, void* stream) {
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, axis, blk, qtype, q_out, ld_q, scales_out);
+  if (st != HALO_OK) return st;
+  if (group != 64 && group != 128) return HALO_ERR_BLOCK;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (axis == HALO_AXIS_COLS) {
+    RotqExtras ex;
+    ex.signs = nullptr;
+    ex.rand = nullptr;
+    ex.ld_rand = 0;
+    return launch_rotq_rows(x_bf16, rows, cols, ld_x, blk, qtype, q_out, ld_q, scales_out, ex, false, s, dev,
+                            nullptr, 0, nullptr, group);
+  }
+  return launch_rotq_cols_grouped(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, group, s, dev);
+}
+
+halo_status_t halo_qgemm_grouped(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,
+                                 const float* s_b, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k,
+                                 int group, int qtype, void* c, int otype, int64_t ld_c, void* stream) {
+  halo_status_t st = check_qgemm(a_q, s_a, a_major, ld_a, b_q, s_b, b_major, ld_b, m, n, k, qtype, c, otype, ld_c);
+  if (st != HALO_OK) return st;
+  if (group != 64 && group != 128) return HALO_ERR_BLOCK;
+  if (k % 128 != 0) return HALO_ERR_SHAPE;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  return launch_qgemm_grouped(a_q, s_a, a_major, ld_a, b_q, s_b, b_major, ld_b, m, n, k, group, qtype, c, otype,
+                              ld_c, static_cast<cudaStream_t>(stream), dev);
+}
+
+size_t halo_workspace_size_grouped(int64_t m, int64_t n, int64_t k, int group, int which) {
+  if (m <= 0 || n <= 0 || k <= 0 || (which != 0 && which != 1) || (group != 64 && group != 128)) return 0;
+  return ws_layout(m, n, k, which, which == 0 ? 256 : 128, group).total;
+}
+
 halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,
                          const float* s_b, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k, int qtype,
                          void* c, int otype, int64_t ld_c, void* stream) {
@@ -689,14 +855,31 @@ halo_status_t halo_qgemm(const void* a_q, const float* s_a, int a_major, int64_t
                       static_cast<cudaStream_t>(stream), dev);
 }
 
-halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k, int blk,
-                              int qtype, void* y, int otype, void* ws, size_t ws_bytes, void* stream) {
+// The linear layers with per-row scales (group 0) or group-wise scales.
+static halo_status_t quantize_op(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int axis, int blk,
+                                 int group, int qtype, void* q, int64_t ld_q, float* s, void* stream) {
+  return group ? halo_hadamard_quantize_grouped(x, rows, cols, ld_x, axis, blk, group, qtype, q, ld_q, s, stream)
+               : halo_hadamard_quantize(x, rows, cols, ld_x, axis, blk, qtype, q, ld_q, s, stream);
+}
+
+static halo_status_t gemm_op(const void* a, const float* sa, int a_major, int64_t ld_a, const void* b,
+                             const float* sb, int b_major, int64_t ld_b, int64_t m, int64_t n, int64_t k, int group,
+                             int qtype, void* c, int otype, int64_t ld_c, void* stream) {
+  return group ? halo_qgemm_grouped(a, sa, a_major, ld_a, b, sb, b_major, ld_b, m, n, k, group, qtype, c, otype,
+                                    ld_c, stream)
+               : halo_qgemm(a, sa, a_major, ld_a, b, sb, b_major, ld_b, m, n, k, qtype, c, otype, ld_c, stream);
+}
+
+static halo_status_t linear_fwd_impl(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k,
+                                     int blk, int group, int qtype, void* y, int otype, void* ws, size_t ws_bytes,
+                                     void* stream) {
   if (!x_bf16 || !w_bf16 || !y) return HALO_ERR_NULL;
   if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
   if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
+  if (group != 0 && group != 64 && group != 128) return HALO_ERR_BLOCK;
   if (m <= 0 || n <= 0 || k <= 0 || pad_to(k, blk) > 32768) return HALO_ERR_SHAPE;
   if (!ws) return HALO_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(m, n, k, 0, blk);
+  const WsLayout L = ws_layout(m, n, k, 0, blk, group);
   if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
   const int64_t esz = otype == HALO_OUT_FP32 ? 4 : 2;
   if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y) || !aligned16(ws) || (n * esz) % 16 != 0 ||
@@ -709,9 +892,21 @@ halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m,
   float* sx = reinterpret_cast<float*>(w8 + L.off[2]);
   float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
   halo_status_t st;
-  if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_COLS, blk, qtype, xq, kp, sx, stream)) != HALO_OK) return st;
-  if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_COLS, blk, qtype, wq, kp, sw, stream)) != HALO_OK) return st;
-  return halo_qgemm(xq, sx, HALO_MAJOR_K, kp, wq, sw, HALO_MAJOR_K, kp, m, n, kp, qtype, y, otype, n, stream);
+  if ((st = quantize_op(x_bf16, m, k, k, HALO_AXIS_COLS, blk, group, qtype, xq, kp, sx, stream)) != HALO_OK) return st;
+  if ((st = quantize_op(w_bf16, n, k, k, HALO_AXIS_COLS, blk, group, qtype, wq, kp, sw, stream)) != HALO_OK) return st;
+  return gemm_op(xq, sx, HALO_MAJOR_K, kp, wq, sw, HALO_MAJOR_K, kp, m, n, kp, group, qtype, y, otype, n, stream);
+}
+
+halo_status_t halo_linear_fwd(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k, int blk,
+                              int qtype, void* y, int otype, void* ws, size_t ws_bytes, void* stream) {
+  return linear_fwd_impl(x_bf16, w_bf16, m, n, k, blk, 0, qtype, y, otype, ws, ws_bytes, stream);
+}
+
+halo_status_t halo_linear_fwd_grouped(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k,
+                                      int blk, int group, int qtype, void* y, int otype, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  if (group != 64 && group != 128) return HALO_ERR_BLOCK;
+  return linear_fwd_impl(x_bf16, w_bf16, m, n, k, blk, group, qtype, y, otype, ws, ws_bytes, stream);
 }
 
 halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n, int64_t k,
@@ -737,19 +932,20 @@ halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, in
                          HALO_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
-                              int64_t k, int blk, int qtype, void* dx, int otype_dx, void* dw, int otype_dw,
-                              void* ws, size_t ws_bytes, void* stream) {
+static halo_status_t linear_bwd_impl(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m,
+                                     int64_t n, int64_t k, int blk, int group, int qtype, void* dx, int otype_dx,
+                                     void* dw, int otype_dw, void* ws, size_t ws_bytes, void* stream) {
   if (!dy_bf16 || (!dx && !dw)) return HALO_ERR_NULL;
   if (dx && !w_bf16) return HALO_ERR_NULL;
   if (dw && !x_bf16) return HALO_ERR_NULL;
   if (!valid_qtype(qtype) || (dx && !valid_otype(otype_dx)) || (dw && !valid_otype(otype_dw))) return HALO_ERR_DTYPE;
   if (blk != 128) return HALO_ERR_BLOCK;
+  if (group != 0 && group != 64 && group != 128) return HALO_ERR_BLOCK;
   if (m <= 0 || n <= 0 || k <= 0) return HALO_ERR_SHAPE;
   if (dx && (pad_to(n, blk) > 32768 || k % 16 != 0)) return HALO_ERR_SHAPE;
   if (dw && (n % 16 != 0 || k % 16 != 0)) return HALO_ERR_SHAPE;
   if (!ws) return HALO_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(m, n, k, 1, blk);
+  const WsLayout L = ws_layout(m, n, k, 1, blk, group);
   if (ws_bytes < L.total) return HALO_ERR_WORKSPACE;
   if (!aligned16(dy_bf16) || (x_bf16 && !aligned16(x_bf16)) || (w_bf16 && !aligned16(w_bf16)) ||
       (dx && !aligned16(dx)) || (dw && !aligned16(dw)) || !aligned16(ws))
@@ -766,12 +962,12 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
     float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
     // dX[M,K] = dY[M,N] W[N,K]: contraction over N (zero-padded to np).
     const int64_t np = pad_to(n, blk);
-    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, qtype, dyq, np, sdy, stream)) != HALO_OK)
+    if ((st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, group, qtype, dyq, np, sdy, stream)) != HALO_OK)
       return st;
-    if ((st = halo_hadamard_quantize(w_bf16, n, k, k, HALO_AXIS_ROWS, blk, qtype, wq, k, sw, stream)) != HALO_OK)
+    if ((st = quantize_op(w_bf16, n, k, k, HALO_AXIS_ROWS, blk, group, qtype, wq, k, sw, stream)) != HALO_OK)
       return st;
-    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_K, np, wq, sw, HALO_MAJOR_MN, k, m, k, np, qtype, dx, otype_dx, k,
-                         stream)) != HALO_OK)
+    if ((st = gemm_op(dyq, sdy, HALO_MAJOR_K, np, wq, sw, HALO_MAJOR_MN, k, m, k, np, group, qtype, dx, otype_dx, k,
+                      stream)) != HALO_OK)
       return st;
   }
   if (dw) {
@@ -781,15 +977,30 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
     float* sx = reinterpret_cast<float*>(w8 + L.off[7]);
     // dW[N,K] = dY^T[N,M] X[M,K]: contraction over M (tokens, zero-padded to mp).
     const int64_t mp = pad_to(m, blk);
-    if ((st = halo_hadamard_quantize(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, qtype, dyq, n, sdy, stream)) != HALO_OK)
+    if ((st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, group, qtype, dyq, n, sdy, stream)) != HALO_OK)
       return st;
-    if ((st = halo_hadamard_quantize(x_bf16, m, k, k, HALO_AXIS_ROWS, blk, qtype, xq, k, sx, stream)) != HALO_OK)
+    if ((st = quantize_op(x_bf16, m, k, k, HALO_AXIS_ROWS, blk, group, qtype, xq, k, sx, stream)) != HALO_OK)
       return st;
-    if ((st = halo_qgemm(dyq, sdy, HALO_MAJOR_MN, n, xq, sx, HALO_MAJOR_MN, k, n, k, mp, qtype, dw, otype_dw, k,
-                         stream)) != HALO_OK)
+    if ((st = gemm_op(dyq, sdy, HALO_MAJOR_MN, n, xq, sx, HALO_MAJOR_MN, k, n, k, mp, group, qtype, dw, otype_dw, k,
+                      stream)) != HALO_OK)
       return st;
   }
   return HALO_OK;
+}
+
+halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
+                              int64_t k, int blk, int qtype, void* dx, int otype_dx, void* dw, int otype_dw,
+                              void* ws, size_t ws_bytes, void* stream) {
+  return linear_bwd_impl(dy_bf16, x_bf16, w_bf16, m, n, k, blk, 0, qtype, dx, otype_dx, dw, otype_dw, ws, ws_bytes,
+                         stream);
+}
+
+halo_status_t halo_linear_bwd_grouped(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m,
+                                      int64_t n, int64_t k, int blk, int group, int qtype, void* dx, int otype_dx,
+                                      void* dw, int otype_dw, void* ws, size_t ws_bytes, void* stream) {
+  if (group != 64 && group != 128) return HALO_ERR_BLOCK;
+  return linear_bwd_impl(dy_bf16, x_bf16, w_bf16, m, n, k, blk, group, qtype, dx, otype_dx, dw, otype_dw, ws,
+                         ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -1,0 +1,319 @@
+// qgemm_grouped.cuh -- low-precision GEMM on codes with group-wise scales along
+// the contraction dimension:
+//
+//     C[i, j] = sum_G s_a[i, G] * s_b[j, G] * sum_{k in group G} A[i, k] B[j, k]
+//
+// Groups of `group` (64 or 128) consecutive K positions, each with its own
+// scale per operand row (QWHA page sec. 3.1, group_quantize; sec. 3.2: group
+// size 64).  A group's partial product cannot be scaled inside the tensor
+// core, so each group is accumulated on its own and promoted:
+//
+//   warp 0      TMA producer: 128 x 128 A and B tiles (K block of 128 codes,
+//               128-byte swizzle) into a 6-stage ring.
+//   warp 1      tensor-memory allocator and MMA issuer: for every group, the
+//               group's K steps (group / 32 MMAs of 128x128x32) into one of
+//               four 128-column partial accumulators in tensor memory, then a
+//               commit that marks that partial full.
+//   warps 2-9   promotion: eight warps, two per tensor-memory lane quarter;
+//               each thread owns 64 columns of one tile row and keeps their fp32
+//               running sums in registers.  Per group it reads its slice of the
+//               partial (tcgen05.ld), converts it (INT8: exact int32 -> fp32
+//               through the 1.5 * 2^23 offset, |partial| <= 127^2 * 128 < 2^22),
+//               multiplies by s_a[i, G] * s_b[j, G] and adds, then frees the
+//               partial.  The promotion costs a few CUDA-core instructions per
+//               element per group, so it needs many warps to hide its latencies;
+//               the four partials let the MMAs run up to three groups ahead.
+// After the last group the running sums are stored as fp32 or bf16.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "qgemm.cuh"
+
+namespace halo {
+
+enum : unsigned int {
+  kSiteGgProducer = 0x311,
+  kSiteGgMma = 0x312,
+  kSiteGgPartial = 0x313,
+  kSiteGgPromote = 0x314,
+};
+
+constexpr int kGgBM = 128;
+constexpr int kGgBN = 128;
+constexpr int kGgBK = 128;
+constexpr int kGgStages = 6;
+constexpr int kGgABytes = kGgBM * kGgBK;  // 16 KB
+constexpr int kGgBBytes = kGgBN * kGgBK;  // 16 KB
+constexpr int kGgPartials = 4;            // 128-column partial accumulators
+constexpr uint32_t kGgTmemCols = 512;
+constexpr int kGgPromWarps = 8;                      // a multiple of 4 (lane quarters)
+constexpr int kGgThreads = 64 + 32 * kGgPromWarps;  // producer, MMA, promotion
+constexpr int kGgPromThreads = 32 * kGgPromWarps;
+constexpr int kGgColsPerThread = kGgBN * 4 / kGgPromWarps;  // columns of a tile row per promotion thread
+// Dynamic shared memory: stages + 1 KB alignment slack + s_b staging (2 x 128
+// floats) + barriers.
+constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 1024 + 256;
+
+struct GroupedGemmParams {
+  int m, n, k, group;
+  int tiles_m, tiles_n, num_tiles;
+  int a_mn, b_mn;  // operand storage: 0 = K-major, 1 = MN-major
+  uint32_t idesc;
+  // Scale of (row i, group G): sa[i * sa_row + G * sa_grp] (likewise sb).
+  const float* sa;
+  int64_t sa_row, sa_grp;
+  const float* sb;
+  int64_t sb_row, sb_grp;
+  void* c;
+  int64_t ldc;
+  int out_bf16;
+};
+
+template <int QT>
+__global__ void __launch_bounds__(kGgThreads, 1)
+    qgemm_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                         GroupedGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kGgStages * kGgABytes;
+  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // [2][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * kGgBN);
+  uint64_t* empty = full + kGgStages;
+  uint64_t* pfull = empty + kGgStages;
+  uint64_t* pempty = pfull + kGgPartials;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + kGgPartials);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGgStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < kGgPartials; ++b) {
+      mbar_init(&pfull[b], 1);
+      mbar_init(&pempty[b], kGgPromWarps);  // one arrival per promotion warp
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kGgTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kblocks = p.k / kGgBK;            // K is a multiple of 128
+  const int gpb = kGgBK / p.group;            // groups per K block: 1 or 2
+  const int steps_per_group = p.group / 32;   // MMAs (K = 32 each) per group
+  griddep_wait();  // codes and scales written, output read, by the previous kernels
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        int tm, tn;
+        gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, kSiteGgProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], kGgABytes + kGgBBytes);
+          uint8_t* a_dst = sA + stage * kGgABytes;
+          uint8_t* b_dst = sB + stage * kGgBBytes;
+          if (p.a_mn)
+            tma_load_2d(a_dst, &tm_a, &full[stage], tm * kGgBM, kb * kGgBK);
+          else
+            tma_load_2d(a_dst, &tm_a, &full[stage], kb * kGgBK, tm * kGgBM);
+          if (p.b_mn)
+            tma_load_2d(b_dst, &tm_b, &full[stage], tn * kGgBN, kb * kGgBK);
+          else
+            tma_load_2d(b_dst, &tm_b, &full[stage], kb * kGgBK, tn * kGgBN);
+          if (++stage == kGgStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t gi = 0;  // groups issued so far (all tiles)
+      const uint32_t a_step = p.a_mn ? 32u * 128u : 32u;
+      const uint32_t b_step = p.b_mn ? 32u * 128u : 32u;
+      const uint32_t a_lbo = p.a_mn ? static_cast<uint32_t>(kGgBK * 128) : 16u;
+      const uint32_t b_lbo = p.b_mn ? static_cast<uint32_t>(kGgBK * 128) : 16u;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < kblocks && ok; ++kb) {
+          if (!mbar_wait(&full[stage], phase, kSiteGgMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * kGgABytes);
+          const uint32_t b_base = smem_u32(sB + stage * kGgBBytes);
+          for (int gs = 0; gs < gpb; ++gs, ++gi) {
+            const uint32_t pb = gi % kGgPartials;
+            if (!mbar_wait(&pempty[pb], ((gi / kGgPartials) & 1u) ^ 1u, kSiteGgPartial)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + pb * 128u;
+            for (int kk = 0; kk < steps_per_group; ++kk) {
+              const int ks = gs * steps_per_group + kk;  // K step (of 32) inside the block
+              const uint64_t adesc = smem_desc_sw128(a_base + ks * a_step, a_lbo, 1024u);
+              const uint64_t bdesc = smem_desc_sw128(b_base + ks * b_step, b_lbo, 1024u);
+              if (QT == 0)
+                mma_i8(d_tmem, adesc, bdesc, p.idesc, kk > 0 ? 1u : 0u);
+              else
+                mma_f8(d_tmem, adesc, bdesc, p.idesc, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&pfull[pb]);  // this group's partial is complete
+          }
+          mma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == kGgStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // Promotion.  A warp may only read tensor-memory lanes 32*(warp%4) .. +31:
+    // that quarter gives the tile rows, (warp - 2) / 4 the 32-column slice.
+    const int quad = warp & 3;
+    const int slice = (warp - 2) >> 2;  // this thread's kGgColsPerThread-column slice
+    const int row_in_tile = quad * 32 + lane;
+    const int ngroups = p.k / p.group;
+    // s_b staging: the 128 threads of the first four promotion warps each load
+    // one column's scale per group into shared memory.
+    const bool stager = (warp - 2) < 4;
+    const int scol_in_tile = (warp - 2) * 32 + lane;  // valid for stagers: 0..127
+    uint32_t gi = 0;
+    bool dead = false;
+    for (int tile = blockIdx.x; tile < p.num_tiles && !dead; tile += gridDim.x) {
+      int tm, tn;
+      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+      const int row = tm * kGgBM + row_in_tile;
+      const bool row_ok = row < p.m;
+      const int scol = tn * kGgBN + scol_in_tile;
+      const bool scol_ok = stager && scol < p.n;
+      const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_row;
+      const float* sb_col = p.sb + static_cast<int64_t>(scol_ok ? scol : 0) * p.sb_row;
+      float sa_next = row_ok ? __ldg(sa_row) : 0.f;
+      float sb_next = scol_ok ? __ldg(sb_col) : 0.f;
+      float run[kGgColsPerThread];
+#pragma unroll
+      for (int j = 0; j < kGgColsPerThread; ++j) run[j] = 0.f;
+      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + slice * kGgColsPerThread;
+#pragma unroll 1
+      for (int g = 0; g < ngroups; ++g, ++gi) {
+        // Alternate by the running group count (not g): consecutive groups use
+        // different buffers across tile boundaries too, so a buffer is only
+        // rewritten after every thread has passed the barrier of the group
+        // after the one that last read it.
+        float* sb_buf = sbuf + (gi & 1u) * kGgBN;
+        if (stager) sb_buf[scol_in_tile] = sb_next;
+        const float sa = sa_next;
+        if (g + 1 < ngroups) {  // next group's scales, loaded early
+          sa_next = row_ok ? __ldg(sa_row + static_cast<int64_t>(g + 1) * p.sa_grp) : 0.f;
+          if (stager) sb_next = scol_ok ? __ldg(sb_col + static_cast<int64_t>(g + 1) * p.sb_grp) : 0.f;
+        }
+        const uint32_t pb = gi % kGgPartials;
+        // One warp per lane quarter polls the partial's barrier; the others
+        // sleep in the named barrier below instead of spinning.
+        const bool ok = slice != 0 || mbar_wait(&pfull[pb], (gi / kGgPartials) & 1u, kSiteGgPromote);
+        // All promotion threads: the partial is complete, sb_buf is published,
+        // and a wait that ran out stops all.
+        if (bar_or(1, kGgPromThreads, !ok)) { dead = true; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < kGgColsPerThread / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_cols + pb * 128u + ch * 32, r);
+        tmem_ld_wait();
+        if (ch == kGgColsPerThread / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[pb]);  // the partial is in registers: free it early
+        }
+        const float4* sbv4 = reinterpret_cast<const float4*>(sb_buf + slice * kGgColsPerThread + ch * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 sbq = sbv4[q];
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int j = 4 * q + e;
+            const int jr = ch * 32 + j;  // index into run[]
+            float2 a;
+            if (QT == 0) {
+              // exact int32 -> fp32 for |x| < 2^22: the bits of 1.5 * 2^23 + x, minus 1.5 * 2^23
+              a = make_float2(__int_as_float(static_cast<int>(r[j]) + 0x4B400000),
+                              __int_as_float(static_cast<int>(r[j + 1]) + 0x4B400000));
+              a = __fadd2_rn(a, make_float2(-12582912.0f, -12582912.0f));
+            } else {
+              a = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+            }
+            const float2 w = __fmul2_rn(make_float2(sa, sa), e == 0 ? make_float2(sbq.x, sbq.y)
+                                                                      : make_float2(sbq.z, sbq.w));
+            const float2 acc = __ffma2_rn(a, w, make_float2(run[jr], run[jr + 1]));
+            run[jr] = acc.x;
+            run[jr + 1] = acc.y;
+          }
+        }
+        }
+      }
+      if (dead) break;
+      // Store this thread's columns of the tile row, 32 at a time.
+#pragma unroll
+      for (int ch = 0; ch < kGgColsPerThread / 32; ++ch) {
+      const int col0 = tn * kGgBN + slice * kGgColsPerThread + ch * 32;
+      const float* run32 = run + ch * 32;
+      if (row_ok && col0 < p.n) {
+        if (p.out_bf16) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.n) {
+            uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(run32[8 * q + 2 * e], run32[8 * q + 2 * e + 1]);
+                w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              o4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.n) out[j] = __float2bfloat16_rn(run32[j]);
+          }
+        } else {
+          float* out = static_cast<float*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.n) {
+            float4* o4 = reinterpret_cast<float4*>(out);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o4[q] = make_float4(run32[4 * q], run32[4 * q + 1], run32[4 * q + 2], run32[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.n) out[j] = run32[j];
+          }
+        }
+      }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kGgTmemCols);
+  }
+}
+
+}  // namespace halo

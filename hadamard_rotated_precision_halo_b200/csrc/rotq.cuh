@@ -89,6 +89,24 @@ __device__ __forceinline__ float absmax128(const float2 (&v)[64]) {
   return m[0];
 }
 
+// max |v| over elements 0..63 (x) and 64..127 (y) of 128 values held as 64
+// float2 pairs, as two trees.
+__device__ __forceinline__ float2 absmax128_halves(const float2 (&v)[64]) {
+  float m[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    m[i] = fmaxf(fmaxf(fabsf(v[2 * i].x), fabsf(v[2 * i].y)), fmaxf(fabsf(v[2 * i + 1].x), fabsf(v[2 * i + 1].y)));
+#pragma unroll
+  for (int w = 8; w >= 1; w /= 2) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      m[i] = fmaxf(m[i], m[i + w]);
+      m[16 + i] = fmaxf(m[16 + i], m[16 + i + w]);
+    }
+  }
+  return make_float2(m[0], m[16]);
+}
+
 // Column-wise max |v| of 64 float2 (x and y are two columns), as trees.
 __device__ __forceinline__ float2 absmax64_cols(const float2 (&v)[64]) {
   float mx[32], my[32];
@@ -203,6 +221,7 @@ struct RotqRowsParams {
   RotqExtras ex;     // EXT = 1 only
   float* scales2;    // QT = 2 only: the E4M3 scales (`scales` holds the INT8 ones)
   float scale_mult2; // QT = 2 only: 1 / (448 * sqrt(blk))
+  int group;         // GR = 1 only: elements per scale group (64 or 128), scales [rows][nb * 128 / group]
 };
 
 // QT = 2: both code sets from one read of the input -- INT8 codes with their
@@ -228,7 +247,9 @@ __device__ __forceinline__ void group_sync(int gw, int grp) {
 
 // PAD = 1: the row length is not a multiple of the block (zero padding); the
 // instantiation for whole blocks (PAD = 0) carries none of that logic.
-template <int BLK, int QT, int EXT, int PAD>
+// GR = 1: group-wise scales, one per p.group (64 or 128) consecutive elements
+// of a row instead of one per row (QT 0 / 1, EXT 0 only).
+template <int BLK, int QT, int EXT, int PAD, int GR = 0>
 __global__ void __launch_bounds__(256)
     rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xt,
                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
@@ -343,6 +364,39 @@ __global__ void __launch_bounds__(256)
         v[i] = upper ? f2_sub(o, v[i]) : f2_add(v[i], o);
       }
     }
+    if (GR) {
+      // Group-wise scales: every group lies inside one thread's 128-element
+      // chunk, so no reduction crosses threads.
+      const float2 hm = absmax128_halves(v);
+      const bool g64 = p.group == 64;
+      const float a0 = g64 ? hm.x : fmaxf(hm.x, hm.y);
+      const float a1 = g64 ? hm.y : a0;
+      const float r0 = a0 > 0.f ? __fdiv_rn(p.qmax, a0) : 0.f;
+      const float r1 = a1 > 0.f ? __fdiv_rn(p.qmax, a1) : 0.f;
+      group_sync(gw, grp);  // orders the leader's store wait before the code writes
+      if (is_active) {
+        const int gpc = g64 ? 2 : 1;  // scale groups per 128-element chunk
+        float* srow = p.scales + row * static_cast<int64_t>(p.nb) * gpc + chunk * gpc;
+        srow[0] = a0 * p.scale_mult;
+        if (g64) srow[1] = a1 * p.scale_mult;
+        uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float r = k < 4 ? r0 : r1;  // elements 16k .. 16k + 15
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = v[8 * k + 2 * j];
+            const float2 b = v[8 * k + 2 * j + 1];
+            if (QT == 0)
+              w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r), q_int8_bits(b.y, r));
+            else
+              w[j] = e4m3x2_bits(a.x * r, a.y * r) | (e4m3x2_bits(b.x * r, b.y * r) << 16);
+          }
+          dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    } else {
     const float amax = absmax128(v);
     uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if (gw > 1) {
@@ -430,6 +484,7 @@ __global__ void __launch_bounds__(256)
       }
       }
     }
+    }  // GR
     fence_proxy_async_smem();
     group_sync(gw, grp);
     if (leader) {
@@ -485,48 +540,54 @@ __device__ __forceinline__ void cols_fwht_rest(float2 (&v)[64]) {
   }
 }
 
-// Codes of the lane's 64 rows x 2 columns into a [128][32]-byte tile.
-// `rnd` (EXT only): random bits of this lane's two columns in the block's
-// first row (stride ld_rand between rows), or nullptr for round to nearest.
+// Codes of 16 of the lane's rows (v16[i] is row 2 (i0 + i) + h, two columns)
+// into a [128][32]-byte tile.  `rnd` (EXT only): random bits of this lane's
+// two columns in the block's first row (stride ld_rand between rows), or
+// nullptr for round to nearest.
 template <int QT, int EXT = 0>
-__device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
-                                                 int h, const uint16_t* rnd = nullptr, int64_t ld_rand = 0) {
+__device__ __forceinline__ void cols_write_codes16(uint8_t* tile, const float2* v16, int i0, float r0, float r1,
+                                                   int pcol, int h, const uint16_t* rnd, int64_t ld_rand) {
   uint16_t* outw = reinterpret_cast<uint16_t*>(tile);
   if (EXT && rnd != nullptr) {
-    // Random bits in batches of 16 rows, loaded before the code stores so that
-    // the loads overlap instead of waiting one by one behind each store.
+    // The 16 rows' random bits are loaded before the code stores so that the
+    // loads overlap instead of waiting one by one behind each store.
+    uint32_t rb[16];
 #pragma unroll
-    for (int i0 = 0; i0 < 64; i0 += 16) {
-      uint32_t rb[16];
+    for (int i = 0; i < 16; ++i)
+      rb[i] = __ldg(reinterpret_cast<const uint32_t*>(rnd + (2 * (i0 + i) + h) * ld_rand));
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        rb[i] = __ldg(reinterpret_cast<const uint32_t*>(rnd + (2 * (i0 + i) + h) * ld_rand));
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float u0 = rand_unit(rb[i] & 0xFFFFu), u1 = rand_unit(rb[i] >> 16);
-        const float2 x = v[i0 + i];
-        uint32_t code;
-        if (QT == 0)
-          code = __byte_perm(q_int8_sr(x.x * r0, u0), q_int8_sr(x.y * r1, u1), 0x0040) & 0xFFFFu;
-        else
-          code = e4m3x2_bits(e4m3_sr_value(x.x * r0, u0), e4m3_sr_value(x.y * r1, u1));
-        outw[(2 * (i0 + i) + h) * 16 + pcol] = static_cast<uint16_t>(code);
-      }
+    for (int i = 0; i < 16; ++i) {
+      const float u0 = rand_unit(rb[i] & 0xFFFFu), u1 = rand_unit(rb[i] >> 16);
+      const float2 x = v16[i];
+      uint32_t code;
+      if (QT == 0)
+        code = __byte_perm(q_int8_sr(x.x * r0, u0), q_int8_sr(x.y * r1, u1), 0x0040) & 0xFFFFu;
+      else
+        code = e4m3x2_bits(e4m3_sr_value(x.x * r0, u0), e4m3_sr_value(x.y * r1, u1));
+      outw[(2 * (i0 + i) + h) * 16 + pcol] = static_cast<uint16_t>(code);
     }
     return;
   }
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
+  for (int i = 0; i < 16; ++i) {
     uint32_t code;
     if (QT == 0) {
       // Both columns in one packed FMA (same rounding as q_int8_bits).
-      const float2 t = __ffma2_rn(v[i], make_float2(r0, r1), make_float2(12582912.0f, 12582912.0f));
+      const float2 t = __ffma2_rn(v16[i], make_float2(r0, r1), make_float2(12582912.0f, 12582912.0f));
       code = __byte_perm(__float_as_uint(t.x), __float_as_uint(t.y), 0x0040);  // low 16 bits stored
     } else {
-      code = e4m3x2_bits(v[i].x * r0, v[i].y * r1);
+      code = e4m3x2_bits(v16[i].x * r0, v16[i].y * r1);
     }
-    outw[(2 * i + h) * 16 + pcol] = static_cast<uint16_t>(code);
+    outw[(2 * (i0 + i) + h) * 16 + pcol] = static_cast<uint16_t>(code);
   }
+}
+
+// Codes of all of the lane's 64 rows x 2 columns.
+template <int QT, int EXT = 0>
+__device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
+                                                 int h, const uint16_t* rnd = nullptr, int64_t ld_rand = 0) {
+#pragma unroll
+  for (int i0 = 0; i0 < 64; i0 += 16) cols_write_codes16<QT, EXT>(tile, v + i0, i0, r0, r1, pcol, h, rnd, ld_rand);
 }
 
 struct RotqColsParams {
@@ -843,6 +904,153 @@ __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
   __syncthreads();
   cluster_arrive();  // no CTA leaves while a peer could still store into its shared memory
   cluster_wait();
+}
+
+// ------------------------------------------------------------------------------------------
+// rotq_cols_grouped: rotation along dimension 0 with group-wise scales, one per
+// `group` (64 or 128) consecutive rows of a column.  A group never leaves a
+// 128-row block, so every warp works alone: persistent warps walk the (block,
+// strip) items in order, each a 128 x 32 tile brought in by TMA through a
+// two-stage ring per warp, rotated in registers (lane layout of
+// cols_load_fwht), its group maxima taken over the two lanes that share a
+// column pair, and its codes written into the consumed stage and stored by TMA.
+// ------------------------------------------------------------------------------------------
+struct RotqColsGrParams {
+  float* scales;  // [rows_p / group][cols]
+  int64_t cols;
+  int strips;     // ceil(cols / 32)
+  int nblocks;    // rows_p / 128
+  int group;      // 64 or 128
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(128))
+};
+
+enum : unsigned int { kSiteRotqColsGrLoad = 0x204 };
+
+// Column-wise max |v| over 32 float2 (x and y are two columns), as trees.
+__device__ __forceinline__ float2 absmax32_cols(const float2* v) {
+  float mx[16], my[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    mx[i] = fmaxf(fabsf(v[2 * i].x), fabsf(v[2 * i + 1].x));
+    my[i] = fmaxf(fabsf(v[2 * i].y), fabsf(v[2 * i + 1].y));
+  }
+#pragma unroll
+  for (int w = 8; w >= 1; w /= 2) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      mx[i] = fmaxf(mx[i], mx[i + w]);
+      my[i] = fmaxf(my[i], my[i + w]);
+    }
+  }
+  return make_float2(mx[0], my[0]);
+}
+
+template <int QT>
+__global__ void __launch_bounds__(128, 3)
+    rotq_cols_grouped_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                             RotqColsGrParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t bars[4][2];
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int pcol = lane & 15;
+  const int h = lane >> 4;
+  uint8_t* s_in = smem + warp * (2 * kColsInBytes);
+
+  if (lane == 0) {
+    mbar_init(&bars[warp][0], 1);
+    mbar_init(&bars[warp][1], 1);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const int64_t items = static_cast<int64_t>(p.nblocks) * p.strips;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * 4;
+  const int64_t nmine = wid < items ? (items - wid + nw - 1) / nw : 0;
+
+  auto issue = [&](int64_t k) {
+    const int64_t it = wid + k * nw;
+    const int b = static_cast<int>(it / p.strips), sidx = static_cast<int>(it % p.strips);
+    const int st = static_cast<int>(k & 1);
+    mbar_arrive_expect_tx(&bars[warp][st], kColsInBytes);
+    tma_load_2d(s_in + st * kColsInBytes, &tm_x, &bars[warp][st], sidx * kColsStrip, b * 128);
+  };
+  if (lane == 0) {
+    if (nmine > 0) issue(0);
+    if (nmine > 1) issue(1);
+  }
+
+  const bool g64 = p.group == 64;
+  bool dead = false;  // a load wait ran out: stop waiting and loading
+  for (int64_t k = 0; k < nmine; ++k) {
+    const int par = static_cast<int>(k & 1);
+    const int64_t it = wid + k * nw;
+    const int b = static_cast<int>(it / p.strips);
+    const int c0 = static_cast<int>(it % p.strips) * kColsStrip;
+    float2 v[64];
+    if (!dead) {
+      const bool ok = mbar_wait(&bars[warp][par], static_cast<uint32_t>((k >> 1) & 1), kSiteRotqColsGrLoad);
+      dead = __any_sync(0xffffffffu, !ok);
+    }
+    if (!dead) {
+      cols_load_fwht<0>(reinterpret_cast<const uint32_t*>(s_in + par * kColsInBytes), pcol, h, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
+    }
+    __syncwarp();
+    cols_fwht_rest(v);
+    // The other stage held item k - 1, whose codes were stored from it at the
+    // end of the previous iteration: once that store has read them, refill it.
+    if (lane == 0 && !dead && k >= 1 && k + 1 < nmine) {
+      bulk_wait_read<0>();
+      issue(k + 1);
+    }
+    // Rows 0..63 of the block are the lane's pairs 0..31, rows 64..127 pairs 32..63.
+    float2 lo = absmax32_cols(v), hi = absmax32_cols(v + 32);
+    lo.x = fmaxf(lo.x, __shfl_xor_sync(0xffffffffu, lo.x, 16));
+    lo.y = fmaxf(lo.y, __shfl_xor_sync(0xffffffffu, lo.y, 16));
+    hi.x = fmaxf(hi.x, __shfl_xor_sync(0xffffffffu, hi.x, 16));
+    hi.y = fmaxf(hi.y, __shfl_xor_sync(0xffffffffu, hi.y, 16));
+    if (!g64) {
+      lo = make_float2(fmaxf(lo.x, hi.x), fmaxf(lo.y, hi.y));
+      hi = lo;
+    }
+    const float rl0 = lo.x > 0.f ? __fdiv_rn(p.qmax, lo.x) : 0.f, rl1 = lo.y > 0.f ? __fdiv_rn(p.qmax, lo.y) : 0.f;
+    const float rh0 = hi.x > 0.f ? __fdiv_rn(p.qmax, hi.x) : 0.f, rh1 = hi.y > 0.f ? __fdiv_rn(p.qmax, hi.y) : 0.f;
+    const int col = c0 + 2 * pcol;
+    if (h == 0 && col < p.cols) {  // cols % 8 == 0: both columns of the pair are in range
+      if (g64) {
+        float* s0 = p.scales + static_cast<int64_t>(2 * b) * p.cols + col;
+        s0[0] = lo.x * p.scale_mult;
+        s0[1] = lo.y * p.scale_mult;
+        s0[p.cols] = hi.x * p.scale_mult;
+        s0[p.cols + 1] = hi.y * p.scale_mult;
+      } else {
+        float* s0 = p.scales + static_cast<int64_t>(b) * p.cols + col;
+        s0[0] = lo.x * p.scale_mult;
+        s0[1] = lo.y * p.scale_mult;
+      }
+    }
+    uint8_t* s_codes = s_in + par * kColsInBytes;  // every lane has read this stage (warp sync above)
+#pragma unroll
+    for (int c = 0; c < 4; ++c)  // pairs 16c .. 16c + 15 = rows 32c .. 32c + 31
+      cols_write_codes16<QT, 0>(s_codes, v + 16 * c, 16 * c, c < 2 ? rl0 : rh0, c < 2 ? rl1 : rh1, pcol, h,
+                                nullptr, 0);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&tm_q, s_codes, c0, b * 128);
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait<0>();
 }
 
 }  // namespace halo

@@ -207,6 +207,52 @@ halo_status_t halo_linear_bwd(const void* dy_bf16, const void* x_bf16, const voi
                               void* stream);
 
 /*
+ * Group-wise scales (QWHA page sec. 3.1, the quantiser's group_quantize: one
+ * scale max|x| / qmax per group of group_size consecutive values; sec. 3.2
+ * recommends 64, sec. 6 32-128): the variant of the calls above in which each
+ * operand carries one scale per `group` (64 or 128) consecutive positions of
+ * the GEMM's contraction dimension instead of one per row.
+ *
+ * halo_hadamard_quantize_grouped: as halo_hadamard_quantize (zero padding
+ * included), with scales
+ *   HALO_AXIS_COLS: scales_out[rows][cols_p / group] (dense), the scale of
+ *                   elements g*group .. g*group + group - 1 of a row;
+ *   HALO_AXIS_ROWS: scales_out[rows_p / group][cols] (dense), the scale of
+ *                   rows g*group .. of a column.
+ * group in {64, 128}, else HALO_ERR_BLOCK.
+ */
+halo_status_t halo_hadamard_quantize_grouped(const void* x_bf16, int64_t rows, int64_t cols,
+                                             int64_t ld_x, int axis, int blk, int group, int qtype,
+                                             void* q_out, int64_t ld_q, float* scales_out, void* stream);
+
+/*
+ * halo_qgemm_grouped: C[i, j] = sum_G s_a[i, G] s_b[j, G] sum_{k in group G}
+ * A[i, k] B[j, k], K a multiple of 128.  Scale layouts follow the codes: a
+ * K-major operand ([M, K] codes) has scales [M][K / group]; an MN-major one
+ * ([K, M] codes, rotated along dimension 0) has scales [K / group][M] -- the
+ * layouts halo_hadamard_quantize_grouped writes.  Everything else as
+ * halo_qgemm.  Each group's partial product is accumulated exactly (int32 /
+ * fp32 on the tensor cores) and scaled into an fp32 running sum.
+ */
+halo_status_t halo_qgemm_grouped(const void* a_q, const float* s_a, int a_major, int64_t ld_a,
+                                 const void* b_q, const float* s_b, int b_major, int64_t ld_b,
+                                 int64_t m, int64_t n, int64_t k, int group, int qtype, void* c,
+                                 int otype, int64_t ld_c, void* stream);
+
+/* Scratch bytes of halo_linear_fwd_grouped (which = 0) / halo_linear_bwd_grouped (which = 1). */
+size_t halo_workspace_size_grouped(int64_t m, int64_t n, int64_t k, int group, int which);
+
+/* halo_linear_fwd / halo_linear_bwd with group-wise scales along each GEMM's
+ * contraction dimension (group 64 or 128); ws as halo_workspace_size_grouped. */
+halo_status_t halo_linear_fwd_grouped(const void* x_bf16, const void* w_bf16, int64_t m, int64_t n,
+                                      int64_t k, int blk, int group, int qtype, void* y, int otype,
+                                      void* ws, size_t ws_bytes, void* stream);
+halo_status_t halo_linear_bwd_grouped(const void* dy_bf16, const void* x_bf16, const void* w_bf16,
+                                      int64_t m, int64_t n, int64_t k, int blk, int group, int qtype,
+                                      void* dx, int otype_dx, void* dw, int otype_dw, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/*
  * Size of the library-owned scratch array used by halo_linear_fwd_noalloc.
  */
 #define HALO_NOALLOC_SCRATCH_BYTES (64ull << 20) /* 64 MiB */

@@ -161,3 +161,25 @@ def test_hadamard_quantize_dual_host_validation(lib):
     assert call(a2=500, a3=512, a6=504) == SHAPE   # INT8 codes shorter than the padded row (512)
     assert call(a8=MISALIGNED) == ALIGN
     assert call(a9=520) == ALIGN        # E4M3 row stride not a multiple of 16
+
+
+def test_grouped_host_validation(lib):
+    q = lib.halo_hadamard_quantize_grouped
+    assert q(FAKE, 256, 512, 512, 0, 128, 32, 0, FAKE, 512, FAKE, None) == BLOCK     # group not 64 / 128
+    assert q(FAKE, 256, 512, 512, 0, 64, 64, 0, FAKE, 512, FAKE, None) == BLOCK      # rotation block
+    assert q(None, 256, 512, 512, 0, 128, 64, 0, FAKE, 512, FAKE, None) == NULL
+    assert q(FAKE, 256, 512, 512, 0, 128, 64, 0, FAKE, 504, FAKE, None) == SHAPE     # codes shorter than the row
+    g = lib.halo_qgemm_grouped
+    assert g(FAKE, FAKE, 0, 256, FAKE, FAKE, 0, 256, 128, 128, 256, 96, 0, FAKE, 0, 128, None) == BLOCK
+    assert g(FAKE, FAKE, 0, 256, FAKE, FAKE, 0, 256, 128, 128, 192, 64, 0, FAKE, 0, 128, None) == SHAPE  # K % 128
+    assert g(FAKE, None, 0, 256, FAKE, FAKE, 0, 256, 128, 128, 256, 64, 0, FAKE, 0, 128, None) == NULL
+    assert lib.halo_workspace_size_grouped(256, 256, 512, 32, 0) == 0
+    ws = lib.halo_workspace_size_grouped(256, 256, 512, 64, 0)
+    assert ws >= 2 * 256 * 512 + 2 * 4 * 256 * 8
+    f = lib.halo_linear_fwd_grouped
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 32, 0, FAKE, 0, FAKE, ws, None) == BLOCK
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 64, 0, FAKE, 0, FAKE, ws - 1, None) == WORKSPACE
+    b = lib.halo_linear_bwd_grouped
+    wsb = lib.halo_workspace_size_grouped(256, 256, 512, 64, 1)
+    assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 48, 0, FAKE, 0, FAKE, 0, FAKE, wsb, None) == BLOCK
+    assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 64, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE

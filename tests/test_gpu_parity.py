@@ -462,6 +462,87 @@ def test_linear_bwd_padded_n_and_m():
     check_output(dw, oracle.linear_bwd_dw(dy2, x, 128, E4M3))         # M = 1000, padded to 1024
 
 
+# -------------------------------------------------------------- group-wise scales
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols,blk,group", [(300, 640, 128, 64), (300, 640, 128, 128), (130, 512, 256, 64),
+                                                 (5, 1000, 128, 64), (3, 28672, 128, 128)])
+def test_rotq_rows_grouped_parity(qtype, rows, cols, blk, group):
+    x = inputs.activations(rows, cols, seed=rows + 2 * cols + group, device="cpu")
+    x[min(1, rows - 1), :64] = 0  # an all-zero group
+    q, s = halo.halo_hadamard_quantize_grouped(_cuda(x), COLS, blk, group, qtype)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle.quantize_grouped(oracle.rotate(x, blk, 1), 1, group, qtype)
+    assert tuple(s.shape) == scales.shape
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols,group", [(1024, 208, 64), (1024, 208, 128), (1000, 48, 64), (8320, 32, 128),
+                                             (128, 16, 64)])
+def test_rotq_cols_grouped_parity(qtype, rows, cols, group):
+    x = inputs.activations(rows, cols, seed=rows + 3 * cols + group, device="cpu")
+    x[:64, min(3, cols - 1)] = 0  # an all-zero group
+    q, s = halo.halo_hadamard_quantize_grouped(_cuda(x), ROWS, 128, group, qtype)
+    torch.cuda.synchronize()
+    codes, scales, t = oracle.quantize_grouped(oracle.rotate(x, 128, 0), 0, group, qtype)
+    assert tuple(s.shape) == scales.shape
+    check_codes(q, s, codes, scales, t, qtype)
+
+
+def _group_scales(outer, ngroups, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand((outer, ngroups), generator=g) * 1.5 + 0.25).to(torch.float32)
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1), (0, 1), (1, 0)])
+@pytest.mark.parametrize("m,n,k", [(300, 520, 640), (16, 16, 256), (640, 272, 1024)])
+def test_qgemm_grouped_parity(qtype, group, a_major, b_major, m, n, k):
+    """Random codes and group scales; the GPU promotes each group's exact
+    partial product into fp32 running sums, the oracle sums in fp64."""
+    if a_major == 1 and m % 16 or b_major == 1 and n % 16:
+        pytest.skip("MN-major storage needs a 16-byte row stride")
+    a = _rand_codes(m, k, qtype, seed=m + k + group)
+    b = _rand_codes(n, k, qtype, seed=n * 3 + k)
+    sa = _group_scales(m, k // group, seed=m)
+    sb = _group_scales(n, k // group, seed=n + 1)
+    # scale layouts follow the code storage: [outer, K/g] K-major, [K/g, outer] MN-major
+    sa_dev = _cuda(sa if a_major == 0 else sa.t().contiguous())
+    sb_dev = _cuda(sb if b_major == 0 else sb.t().contiguous())
+    c = halo.halo_qgemm_grouped(_cuda(_stored(a, a_major)), sa_dev, a_major, _cuda(_stored(b, b_major)), sb_dev,
+                                b_major, m, n, k, group, qtype, FP32)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_grouped(a.view(torch.uint8).numpy(), sa.numpy(), b.view(torch.uint8).numpy(), sb.numpy(),
+                              group, qtype)
+    err = np.abs(c.cpu().numpy().astype(np.float64) - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("group", [64, 128])
+def test_linear_grouped_parity(qtype, group):
+    m, n, k = 384, 320, 640
+    x = inputs.activations(m, k, seed=71, device="cpu")
+    w = inputs.weights(n, k, seed=72, device="cpu")
+    dy = inputs.grads(m, n, seed=73, device="cpu")
+    y = halo.halo_linear_fwd_grouped(_cuda(x), _cuda(w), 128, group, qtype, FP32)
+    dx, dw = halo.halo_linear_bwd_grouped(_cuda(dy), _cuda(x), _cuda(w), 128, group, qtype, FP32, FP32)
+    torch.cuda.synchronize()
+    check_output(y, oracle.linear_fwd_grouped(x, w, 128, group, qtype))
+    check_output(dx, oracle.linear_bwd_dx_grouped(dy, w, 128, group, qtype))
+    check_output(dw, oracle.linear_bwd_dw_grouped(dy, x, 128, group, qtype))
+
+
+def test_linear_grouped_padded_and_bf16():
+    m, n, k = 200, 136, 1000
+    x = inputs.activations(m, k, seed=74, device="cpu")
+    w = inputs.weights(n, k, seed=75, device="cpu")
+    y = halo.halo_linear_fwd_grouped(_cuda(x), _cuda(w), 128, 64, INT8, BF16)
+    torch.cuda.synchronize()
+    check_output(y, oracle.linear_fwd_grouped(x, w, 128, 64, INT8))
+
+
 # ------------------------------------------------------------------- edge cases
 def test_single_token_forward_and_tiny_backward():
     x = inputs.activations(1, 256, seed=91, device="cpu")
