@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/halo.h"
@@ -31,7 +32,7 @@ thread_local char g_last_detail[256] = "";
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
-  bool ready = false;
+  std::atomic<bool> ready{false};  // set last, with release order, once the rest is filled in
   bool supported = false;
   int sm_count = 0;
 };
@@ -129,9 +130,9 @@ halo_status_t device_setup(int* dev_out) {
   if (dev < 0 || dev >= kMaxDevices) return HALO_ERR_UNSUPPORTED;
   *dev_out = dev;
   DeviceInfo& d = g_dev[dev];
-  if (d.ready) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+  if (d.ready.load(std::memory_order_acquire)) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_dev_mutex);
-  if (d.ready) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
+  if (d.ready.load(std::memory_order_relaxed)) return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
   int major = 0, minor = 0;
   HALO_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
   HALO_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
@@ -183,7 +184,7 @@ halo_status_t device_setup(int* dev_out) {
     HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1>, optin));
   }
-  d.ready = true;
+  d.ready.store(true, std::memory_order_release);
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
 }
 

@@ -275,9 +275,9 @@ halo_status_t halo_linear_bwd_grouped(const void* dy_bf16, const void* x_bf16, c
  *
  * Limits and behaviour:
  *   - Arguments and layout as for halo_linear_fwd.  Sizes whose codes and
- *     scales do not fit (halo_workspace_size(m, n, k, 0) greater than
- *     HALO_NOALLOC_SCRATCH_BYTES) return HALO_ERR_WORKSPACE and launch nothing;
- *     halo_last_error_detail() then gives the bytes needed.
+ *     scales do not fit (more than HALO_NOALLOC_SCRATCH_BYTES; at most
+ *     halo_workspace_size(m, n, k, 0) are needed) return HALO_ERR_WORKSPACE and
+ *     launch nothing; halo_last_error_detail() then gives the bytes needed.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - All calls share the one array, which keeps the last call's contents.
