@@ -17,10 +17,11 @@
 //   warps 2-9   promotion: eight warps, two per tensor-memory lane quarter;
 //               each thread owns 64 columns of one tile row and keeps their fp32
 //               running sums in registers.  Per group it reads its slice of the
-//               partial (tcgen05.ld), converts it (INT8: exact int32 -> fp32
-//               through the 1.5 * 2^23 offset, |partial| <= 127^2 * 128 < 2^22),
-//               multiplies by s_a[i, G] * s_b[j, G] and adds, then frees the
-//               partial.  The promotion costs a few CUDA-core instructions per
+//               partial (tcgen05.ld), converts it (INT8: exact int32 -> fp32,
+//               |partial| <= 127^2 * 128 < 2^24), multiplies by s_a[i, G] *
+//               s_b[j, G] and adds, then frees the partial.  The s_b of 16
+//               groups are staged in shared memory at a time, so the promotion
+//               warps meet at a barrier once per 16 groups.  The promotion costs a few CUDA-core instructions per
 //               element per group, so it needs many warps to hide its latencies;
 //               the four partials let the MMAs run up to three groups ahead.
 // After the last group the running sums are stored as fp32 or bf16.
@@ -52,9 +53,10 @@ constexpr int kGgPromWarps = 8;                      // a multiple of 4 (lane qu
 constexpr int kGgThreads = 64 + 32 * kGgPromWarps;  // producer, MMA, promotion
 constexpr int kGgPromThreads = 32 * kGgPromWarps;
 constexpr int kGgColsPerThread = kGgBN * 4 / kGgPromWarps;  // columns of a tile row per promotion thread
-// Dynamic shared memory: stages + 1 KB alignment slack + s_b staging (2 x 128
-// floats) + barriers.
-constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 1024 + 256;
+constexpr int kGgChunk = 16;  // groups whose s_b are staged together
+// Dynamic shared memory: stages + 1 KB alignment slack + s_b staging (2 x
+// kGgChunk x 128 floats) + barriers.
+constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 2 * kGgChunk * kGgBN * 4 + 256;
 
 struct GroupedGemmParams {
   int m, n, k, group;
@@ -79,8 +81,8 @@ __global__ void __launch_bounds__(kGgThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGgStages * kGgABytes;
-  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // [2][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * kGgBN);
+  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // [2][kGgChunk][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * kGgChunk * kGgBN);
   uint64_t* empty = full + kGgStages;
   uint64_t* pfull = empty + kGgStages;
   uint64_t* pempty = pfull + kGgPartials;
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
     const bool stager = (warp - 2) < 4;
     const int scol_in_tile = (warp - 2) * 32 + lane;  // valid for stagers: 0..127
     uint32_t gi = 0;
+    uint32_t ci = 0;  // s_b chunks staged so far (all tiles): picks the staging buffer
     bool dead = false;
     for (int tile = blockIdx.x; tile < p.num_tiles && !dead; tile += gridDim.x) {
       int tm, tn;
@@ -203,68 +206,70 @@ __global__ void __launch_bounds__(kGgThreads, 1)
       const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_row;
       const float* sb_col = p.sb + static_cast<int64_t>(scol_ok ? scol : 0) * p.sb_row;
       float sa_next = row_ok ? __ldg(sa_row) : 0.f;
-      float sb_next = scol_ok ? __ldg(sb_col) : 0.f;
       float run[kGgColsPerThread];
 #pragma unroll
       for (int j = 0; j < kGgColsPerThread; ++j) run[j] = 0.f;
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + slice * kGgColsPerThread;
 #pragma unroll 1
-      for (int g = 0; g < ngroups; ++g, ++gi) {
-        // Alternate by the running group count (not g): consecutive groups use
-        // different buffers across tile boundaries too, so a buffer is only
-        // rewritten after every thread has passed the barrier of the group
-        // after the one that last read it.
-        float* sb_buf = sbuf + (gi & 1u) * kGgBN;
-        if (stager) sb_buf[scol_in_tile] = sb_next;
-        const float sa = sa_next;
-        if (g + 1 < ngroups) {  // next group's scales, loaded early
-          sa_next = row_ok ? __ldg(sa_row + static_cast<int64_t>(g + 1) * p.sa_grp) : 0.f;
-          if (stager) sb_next = scol_ok ? __ldg(sb_col + static_cast<int64_t>(g + 1) * p.sb_grp) : 0.f;
+      for (int g0 = 0; g0 < ngroups; g0 += kGgChunk, ++ci) {
+        // Stage the chunk's s_b (kGgChunk groups x 128 columns).  A buffer is
+        // rewritten only after every thread has passed the barrier of the
+        // chunk after the one that last read it (chunks alternate buffers by
+        // the running chunk count, also across tiles).
+        float* sb_chunk = sbuf + (ci & 1u) * (kGgChunk * kGgBN);
+        const int gn = min(kGgChunk, ngroups - g0);
+        if (stager) {
+          for (int gg = 0; gg < gn; ++gg)
+            sb_chunk[gg * kGgBN + scol_in_tile] = scol_ok ? __ldg(sb_col + static_cast<int64_t>(g0 + gg) * p.sb_grp) : 0.f;
         }
-        const uint32_t pb = gi % kGgPartials;
-        // One warp per lane quarter polls the partial's barrier; the others
-        // sleep in the named barrier below instead of spinning.
-        const bool ok = slice != 0 || mbar_wait(&pfull[pb], (gi / kGgPartials) & 1u, kSiteGgPromote);
-        // All promotion threads: the partial is complete, sb_buf is published,
-        // and a wait that ran out stops all.
-        if (bar_or(1, kGgPromThreads, !ok)) { dead = true; break; }
-        tc_fence_after();
+        // All promotion threads: publishes sb_chunk; a wait that ran out in
+        // the previous chunk stops all.
+        if (bar_or(1, kGgPromThreads, dead)) { dead = true; break; }
+#pragma unroll 1
+        for (int gg = 0; gg < gn; ++gg, ++gi) {
+          const int g = g0 + gg;
+          const float sa = sa_next;
+          if (g + 1 < ngroups) sa_next = row_ok ? __ldg(sa_row + static_cast<int64_t>(g + 1) * p.sa_grp) : 0.f;
+          const uint32_t pb = gi % kGgPartials;
+          if (!dead && !mbar_wait(&pfull[pb], (gi / kGgPartials) & 1u, kSiteGgPromote)) dead = true;
+          dead = __any_sync(0xffffffffu, dead);
+          if (dead) continue;  // still reach the next chunk barrier
+          tc_fence_after();
+          const float* sb_buf = sb_chunk + gg * kGgBN;
 #pragma unroll
-        for (int ch = 0; ch < kGgColsPerThread / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_cols + pb * 128u + ch * 32, r);
-        tmem_ld_wait();
-        if (ch == kGgColsPerThread / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty[pb]);  // the partial is in registers: free it early
-        }
-        const float4* sbv4 = reinterpret_cast<const float4*>(sb_buf + slice * kGgColsPerThread + ch * 32);
+          for (int ch = 0; ch < kGgColsPerThread / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_cols + pb * 128u + ch * 32, r);
+          tmem_ld_wait();
+          if (ch == kGgColsPerThread / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[pb]);  // the partial is in registers: free it early
+          }
+          const float4* sbv4 = reinterpret_cast<const float4*>(sb_buf + slice * kGgColsPerThread + ch * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 sbq = sbv4[q];
+          for (int q = 0; q < 8; ++q) {
+            const float4 sbq = sbv4[q];
 #pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int j = 4 * q + e;
-            const int jr = ch * 32 + j;  // index into run[]
-            float2 a;
-            if (QT == 0) {
-              // exact int32 -> fp32 for |x| < 2^22: the bits of 1.5 * 2^23 + x, minus 1.5 * 2^23
-              a = make_float2(__int_as_float(static_cast<int>(r[j]) + 0x4B400000),
-                              __int_as_float(static_cast<int>(r[j + 1]) + 0x4B400000));
-              a = __fadd2_rn(a, make_float2(-12582912.0f, -12582912.0f));
-            } else {
-              a = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+            for (int e = 0; e < 4; e += 2) {
+              const int j = 4 * q + e;
+              const int jr = ch * 32 + j;  // index into run[]
+              float2 a;
+              if (QT == 0)
+                a = make_float2(__int2float_rn(static_cast<int>(r[j])), __int2float_rn(static_cast<int>(r[j + 1])));
+              else
+                a = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+              const float2 w = __fmul2_rn(make_float2(sa, sa), e == 0 ? make_float2(sbq.x, sbq.y)
+                                                                        : make_float2(sbq.z, sbq.w));
+              const float2 acc = __ffma2_rn(a, w, make_float2(run[jr], run[jr + 1]));
+              run[jr] = acc.x;
+              run[jr + 1] = acc.y;
             }
-            const float2 w = __fmul2_rn(make_float2(sa, sa), e == 0 ? make_float2(sbq.x, sbq.y)
-                                                                      : make_float2(sbq.z, sbq.w));
-            const float2 acc = __ffma2_rn(a, w, make_float2(run[jr], run[jr + 1]));
-            run[jr] = acc.x;
-            run[jr + 1] = acc.y;
+          }
           }
         }
-        }
       }
+      if (bar_or(1, kGgPromThreads, dead)) dead = true;  // agree before the stores
       if (dead) break;
       // Store this thread's columns of the tile row, 32 at a time.
 #pragma unroll
