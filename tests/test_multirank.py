@@ -61,3 +61,26 @@ def test_reference_arm_on_a_nonzero_rank_exits_without_work():
                           "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
     assert res.returncode == 0
     assert res.stdout.strip() == ""
+
+
+def test_reference_arm_prints_one_contract_line():
+    """rank 0 of the reference arm: the oracle on a bounded sample of the layer
+    step, one JSON line with the keys the bench contract asks for."""
+    import json
+
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["unit"] == "TOPS"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "llama70b_layer_fwd_bwd"
