@@ -53,6 +53,7 @@ EXPORTS = (
     "halo_linear_fwd_noalloc",
     "halo_status_string",
     "halo_device_error",
+    "halo_selftest_wait_timeout",
     "halo_last_cuda_error",
     "halo_last_error_detail",
 )
@@ -97,6 +98,8 @@ def lib():
     L.halo_linear_fwd_grouped.restype = I
     L.halo_linear_bwd_grouped.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I, P, I, P, SZ, P]
     L.halo_linear_bwd_grouped.restype = I
+    L.halo_selftest_wait_timeout.argtypes = [I64, P]
+    L.halo_selftest_wait_timeout.restype = I
     L.halo_qgemm.argtypes = [P, P, I, I64, P, P, I, I64, I64, I64, I64, I, P, I, I64, P]
     L.halo_qgemm.restype = I
     L.halo_workspace_size.argtypes = [I64, I64, I64, I]

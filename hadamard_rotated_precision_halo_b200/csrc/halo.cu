@@ -249,6 +249,21 @@ halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
   return HALO_OK;
 }
 
+// Failure-path self-test: one thread waits, with the given bound, on an
+// mbarrier that nothing ever completes; the wait runs out, records its site
+// in the device error word and returns (no trap, no hang).
+enum : unsigned int { kSiteSelftest = 0xF01 };
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, kSiteSelftest, limit_ns);
+}
+
 // n rounded up to a multiple of b (the zero-padded length of a rotated dimension).
 int64_t pad_to(int64_t n, int64_t b) { return (n + b - 1) / b * b; }
 
@@ -748,6 +763,16 @@ halo_status_t halo_device_error(int* where) {
   if (site != 0) HALO_CUDA(cudaMemcpyToSymbol(g_error_site, &zero, sizeof(zero)));
   if (where) *where = static_cast<int>(site);
   return site ? HALO_ERR_TIMEOUT : HALO_OK;
+}
+
+halo_status_t halo_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns <= 0 || static_cast<unsigned long long>(limit_ns) > kWaitLimitNs) return HALO_ERR_SHAPE;
+  int dev = 0;
+  halo_status_t st = device_setup(&dev);
+  if (st != HALO_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns));
+  HALO_CUDA(cudaGetLastError());
+  return HALO_OK;
 }
 
 size_t halo_workspace_size(int64_t m, int64_t n, int64_t k, int which) {

@@ -64,7 +64,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
 
 // Wait for the phase with parity `phase` to complete.  Bounded: returns false
 // (and records `site`) after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned int site) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, phase)) return true;
   const unsigned long long t0 = globaltimer();
@@ -72,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigne
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, phase)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(site);
       return false;
     }

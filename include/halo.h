@@ -301,6 +301,17 @@ const char* halo_status_string(int status);
  */
 halo_status_t halo_device_error(int* where);
 
+/*
+ * Diagnostic of the failure path (no counterpart in the paper): launches one
+ * kernel that waits, bounded by limit_ns (0 < limit_ns <= 2e9, else
+ * HALO_ERR_SHAPE), on an mbarrier that nothing ever completes.  The wait runs
+ * out, records site 0xF01 in the device error word and returns, exactly as any
+ * other bounded wait in the library does; halo_device_error() then reports
+ * HALO_ERR_TIMEOUT with that site and clears it, and the context stays usable.
+ * Nothing faults, traps or hangs.
+ */
+halo_status_t halo_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 /* The last CUDA error code seen by the library on this thread (0 if none).
  * A failed tensor-map encoding is reported as 10000 + its CUresult. */
 int halo_last_cuda_error(void);

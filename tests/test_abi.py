@@ -183,3 +183,8 @@ def test_grouped_host_validation(lib):
     wsb = lib.halo_workspace_size_grouped(256, 256, 512, 64, 1)
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 48, 0, FAKE, 0, FAKE, 0, FAKE, wsb, None) == BLOCK
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 64, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE
+
+
+def test_selftest_wait_timeout_validation(lib):
+    assert lib.halo_selftest_wait_timeout(0, None) == SHAPE
+    assert lib.halo_selftest_wait_timeout(3_000_000_000, None) == SHAPE
