@@ -11,9 +11,14 @@ gradients N(0, 1e-3^2)); they exceed the 126 MB L2 several times over.
 
 The metric is whole-job throughput in TOPS (2 * M * N * K per GEMM, summed,
 including the rotation and quantisation launches) over the device-timed
-steps; rotate+quantise GB/s and the GEMM kernels' own TOPS are reported beside
-it.  `--impl reference` times the CPU oracle on a bounded sample of the same
-workload instead.
+steps, which replay the step's launches as one captured CUDA graph
+(`--no-graph`: launched from the host); rotate+quantise GB/s and the GEMM
+kernels' own TOPS are reported beside it, and `e2e` times the same step through
+the linear-layer calls with host buffers.  `--qtype e4m3` runs FP8, `--group
+64|128` group-wise scales.  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.  `--measure-peaks` and
+`--rotq-shapes` print the GEMM peak comparison and the per-shape
+rotate+quantise table.
 """
 from __future__ import annotations
 

@@ -1,13 +1,19 @@
 // rotq.cuh -- fused block Walsh-Hadamard rotation + absmax + symmetric quantisation.
 //
-// Two kernels, one per rotation axis of a bf16 matrix X[rows, cols]:
+// Kernels, by rotation axis of a bf16 matrix X[rows, cols]:
 //
-//   rotq_rows_kernel  rotate along the contiguous dimension (blocks of 128 or
-//                     256 consecutive elements of a row), one scale per row.
-//   rotq_cols_kernel  rotate along dimension 0 (blocks of 128 consecutive rows
-//                     of a column), one scale per column.
+//   rotq_rows_kernel        rotate along the contiguous dimension (blocks of
+//                           128 or 256 consecutive elements of a row), one
+//                           scale per row (or per group of 64 / 128 elements).
+//   rotq_cols_1pass_kernel  rotate along dimension 0 (blocks of 128
+//   rotq_cols_kernel        consecutive rows of a column), one scale per
+//                           column: a single pass for up to 8192 rows, two
+//                           passes above.
+//   rotq_cols_grouped_kernel  dimension 0 with one scale per group of 64 / 128
+//                           rows of a column.
+// A rotated length that is not a multiple of the block is zero-padded.
 //
-// Both compute, for every group g (a row or a column),
+// All compute, for every group g (a row, a column or a part of one),
 //     u      = H_blk x            (unnormalised Sylvester transform, fp32)
 //     amax_g = max |u|            (over the whole group)
 //     s_g    = amax_g / (qmax sqrt(blk))        -> scale of the normalised value
@@ -498,7 +504,6 @@ __global__ void __launch_bounds__(256)
 
 constexpr int kColsStrip = 32;
 constexpr int kColsInBytes = 128 * kColsStrip * 2;  // one 128 x 32 bf16 block
-constexpr int kColsOutBytes = 128 * kColsStrip;     // one 128 x 32 block of codes
 constexpr int kColsStages = 2;
 
 // Lane (pcol, h) of a warp owns columns (2 pcol, 2 pcol + 1) and the 64 rows
