@@ -323,7 +323,11 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
     }
   }
   const bool pad = tail != 0 || nbt != nb;
-  const size_t smem = static_cast<size_t>(groups) * rows_group_smem(gw, dual ? 2 : 1, pad) + 128;  // + alignment slack
+  // Code tiles of their own (two rows in flight ahead), or, for one output
+  // when that fits more CTAs on an SM, codes written into the consumed input
+  // stage (one row in flight ahead).
+  const size_t smem_tiles = static_cast<size_t>(groups) * rows_group_smem(gw, dual ? 2 : 1, pad) + 128;  // + alignment slack
+  const size_t smem_in_stage = static_cast<size_t>(groups) * rows_group_smem(gw, 0, pad) + 128;
 
   RotqRowsParams p;
   p.scales = scales;
@@ -341,8 +345,13 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
   p.group = group;
 
   RowsKernel kern = rows_kernel(blk, qtype, ext, pad, group != 0);
-  int per_sm = 0;
-  HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
+  int per_sm = 0, per_sm_in_stage = 0;
+  HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem_tiles));
+  if (!dual) HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_in_stage, kern, threads, smem_in_stage));
+  const bool in_stage = per_sm_in_stage > per_sm;
+  const size_t smem = in_stage ? smem_in_stage : smem_tiles;
+  p.out_tiles = in_stage ? 0 : (dual ? 2 : 1);
+  if (in_stage) per_sm = per_sm_in_stage;
   if (per_sm < 1) per_sm = 1;
   const int64_t ctas_needed = (rows + groups - 1) / groups;
   const int grid = static_cast<int>(std::min<int64_t>(ctas_needed, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));

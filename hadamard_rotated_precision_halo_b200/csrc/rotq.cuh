@@ -228,6 +228,7 @@ struct RotqRowsParams {
   float* scales2;    // QT = 2 only: the E4M3 scales (`scales` holds the INT8 ones)
   float scale_mult2; // QT = 2 only: 1 / (448 * sqrt(blk))
   int group;         // GR = 1 only: elements per scale group (64 or 128), scales [rows][nb * 128 / group]
+  int out_tiles;     // code tiles per row group: 0 (codes written into the consumed input stage), 1, or 2 (QT = 2)
 };
 
 // QT = 2: both code sets from one read of the input -- INT8 codes with their
@@ -235,8 +236,9 @@ struct RotqRowsParams {
 constexpr int kQtDual = 2;
 
 // Shared-memory bytes of one row group: 2 input stages (the per-thread slots,
-// then, when padding, 256 bytes for a partial last chunk) and one code tile
-// (two for the dual output).
+// then, when padding, 256 bytes for a partial last chunk) and `ntiles` code
+// tiles (none when the codes go into the consumed input stage; two for the
+// dual output).
 __host__ __device__ inline uint32_t rows_group_slots_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsInSlot; }
 __host__ __device__ inline uint32_t rows_group_in_bytes(int gw, int pad) { return rows_group_slots_bytes(gw) + (pad ? 256 : 0); }
 __host__ __device__ inline uint32_t rows_group_out_bytes(int gw) { return static_cast<uint32_t>(gw) * 32 * kRowsOutSlot; }
@@ -255,12 +257,18 @@ __device__ __forceinline__ void group_sync(int gw, int grp) {
 // instantiation for whole blocks (PAD = 0) carries none of that logic.
 // GR = 1: group-wise scales, one per p.group (64 or 128) consecutive elements
 // of a row instead of one per row (QT 0 / 1, EXT 0 only).
+// p.out_tiles = 0 (one output, chosen by the launcher when it fits more CTAs
+// on an SM): a row's codes are written into the input stage the row was read
+// from, and that stage is refilled with the next row once their store has read
+// them, so only one row is in flight ahead; with <= 168 registers (the bound
+// below) three 4-warp CTAs of 8192-wide rows fit on an SM.  Otherwise the codes
+// go to tiles of their own and two rows are in flight ahead.
 template <int BLK, int QT, int EXT, int PAD, int GR = 0>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(BLK == 128 && EXT == 0 && QT != kQtDual ? 384 : 256)
     rotq_rows_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xt,
                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
                      RotqRowsParams p) {
-  constexpr int kTiles = QT == kQtDual ? 2 : 1;
+  const bool in_stage = QT != kQtDual && p.out_tiles == 0;  // codes written into the consumed input stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   __shared__ uint64_t full_bar[8][2];
@@ -279,9 +287,9 @@ __global__ void __launch_bounds__(256)
   // One row: the 3-D box of whole chunks, plus the partial chunk's 2-D box.
   const uint32_t in_bytes = PAD ? static_cast<uint32_t>(p.nbt) * kRowsInSlot + (p.tail ? 256u : 0u)
                                : static_cast<uint32_t>(p.nb) * kRowsInSlot;
-  uint8_t* g_in = smem + grp * rows_group_smem(gw, kTiles, PAD);
-  uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw, PAD);
-  uint8_t* g_out2 = g_out + rows_group_out_bytes(gw);  // QT = 2 only
+  uint8_t* g_in = smem + grp * rows_group_smem(gw, p.out_tiles, PAD);
+  uint8_t* g_out = g_in + 2 * rows_group_in_bytes(gw, PAD);  // code tile (unused when in_stage)
+  uint8_t* g_out2 = g_out + rows_group_out_bytes(gw);        // QT = 2 only
 
   if (leader) {
     mbar_init(&full_bar[grp][0], 1);
@@ -355,9 +363,19 @@ __global__ void __launch_bounds__(256)
     }
     group_sync(gw, grp);  // stage `st` fully read
     if (leader) {
-      if (!dead && it + 2 < nmine) issue(it + 2);
-      bulk_wait_read<0>();  // the previous row's store has read the code tile
+      if (in_stage) {
+        // The other stage holds the previous row's codes: once their store
+        // has read them, it takes the next row.
+        if (!dead && it >= 1 && it + 1 < nmine) {
+          bulk_wait_read<0>();
+          issue(it + 1);
+        }
+      } else {
+        if (!dead && it + 2 < nmine) issue(it + 2);
+        bulk_wait_read<0>();  // the previous row's store has read the code tiles
+      }
     }
+    uint8_t* out = in_stage ? g_in + st * rows_group_in_bytes(gw, PAD) : g_out;
     if (BLK == 256) {
       // Top stage of the 256-point transform: chunk pairs (2j, 2j+1) sit on
       // adjacent lanes.  Lower half keeps a + b, upper half a - b.
@@ -379,13 +397,13 @@ __global__ void __launch_bounds__(256)
       const float a1 = g64 ? hm.y : a0;
       const float r0 = a0 > 0.f ? __fdiv_rn(p.qmax, a0) : 0.f;
       const float r1 = a1 > 0.f ? __fdiv_rn(p.qmax, a1) : 0.f;
-      group_sync(gw, grp);  // orders the leader's store wait before the code writes
+      if (!in_stage) group_sync(gw, grp);  // orders the leader's store wait before the code writes
       if (is_active) {
         const int gpc = g64 ? 2 : 1;  // scale groups per 128-element chunk
         float* srow = p.scales + row * static_cast<int64_t>(p.nb) * gpc + chunk * gpc;
         srow[0] = a0 * p.scale_mult;
         if (g64) srow[1] = a1 * p.scale_mult;
-        uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
+        uint4* dst = reinterpret_cast<uint4*>(out + chunk * kRowsOutSlot);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float r = k < 4 ? r0 : r1;  // elements 16k .. 16k + 15
@@ -407,7 +425,7 @@ __global__ void __launch_bounds__(256)
     uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if (gw > 1) {
       if (lane == 0) s_wmax[par][warp] = wmax;
-      group_sync(gw, grp);  // also orders the leader's store wait before the code writes
+      group_sync(gw, grp);  // (code tiles: also orders the leader's store wait before the code writes)
       for (int w = 0; w < gw; ++w) wmax = max(wmax, s_wmax[par][grp * gw + w]);
     } else {
       __syncwarp();
@@ -436,7 +454,7 @@ __global__ void __launch_bounds__(256)
         }
       }
     } else if (is_active) {
-      uint4* dst = reinterpret_cast<uint4*>(g_out + chunk * kRowsOutSlot);
+      uint4* dst = reinterpret_cast<uint4*>(out + chunk * kRowsOutSlot);
       if (EXT && p.ex.rand != nullptr) {
         // Stochastic rounding: the chunk's 128 random values in two batches of
         // 8 vectors, loaded before the code stores so that the loads overlap.
@@ -494,7 +512,7 @@ __global__ void __launch_bounds__(256)
     fence_proxy_async_smem();
     group_sync(gw, grp);
     if (leader) {
-      tma_store_3d(&tm_q, g_out, 0, 0, static_cast<int32_t>(row));
+      tma_store_3d(&tm_q, out, 0, 0, static_cast<int32_t>(row));
       if (QT == kQtDual) tma_store_3d(&tm_q2, g_out2, 0, 0, static_cast<int32_t>(row));
       bulk_commit();  // one group for both stores: the wait above covers both tiles
     }
@@ -637,10 +655,12 @@ __global__ void __launch_bounds__(128, EXT ? 2 : 3)
   const int first = static_cast<int>(crank) + static_cast<int>(csize) * warp;
   const int step = static_cast<int>(csize) * p.warps;
   const int nmine = first < p.nblocks ? (p.nblocks - first + step - 1) / step : 0;
-  const int nseq = 2 * nmine;  // pass 1 then pass 2 over the same blocks
+  // Pass 1 then pass 2 over the same blocks, pass 2 in reverse order: the
+  // blocks read last in pass 1 are the likeliest still to be in L2.
+  const int nseq = 2 * nmine;
 
   auto issue = [&](int j) {
-    const int b = first + step * (j < nmine ? j : j - nmine);
+    const int b = first + step * (j < nmine ? j : 2 * nmine - 1 - j);
     const int s = j % kColsStages;
     mbar_arrive_expect_tx(&bars[warp][s], kColsInBytes);
     tma_load_2d(s_in + s * kColsInBytes, &tm_x, &bars[warp][s], c0, b * 128);
@@ -717,7 +737,7 @@ __global__ void __launch_bounds__(128, EXT ? 2 : 3)
     if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
-    const int bq = first + step * (j - nmine);
+    const int bq = first + step * (2 * nmine - 1 - j);
     cols_load_fwht<EXT>(blkw, pcol, h, v, EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(bq) * 128 : nullptr);
     __syncwarp();
     cols_fwht_rest(v);
