@@ -7,7 +7,8 @@ import oracle
 
 # Quantised codes must match the oracle bit for bit, except where the oracle's
 # pre-rounding value lies within this relative distance of a rounding midpoint
-# (the GPU computes v * (qmax / amax) in fp32; the oracle v / s in fp64).
+# (the GPU computes v * (qmax / amax) in fp32; the oracle v / s in fp64), or
+# within the fp32 transform's own rounding bound of it (rotation_rounding_band).
 BOUNDARY_REL = 1e-6
 # Scales: fp32 on both sides from differently ordered arithmetic.
 SCALE_REL = 1e-6
@@ -19,8 +20,53 @@ def u8(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.uint8).cpu().numpy()
 
 
-def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype):
-    """Returns (#exempt elements, #exempt elements that differ)."""
+def _scale_per_element(scales, shape, axis: int) -> np.ndarray:
+    """Each element's scale: one per row when the blocks run along the
+    contiguous dim (axis 1), one per column when they run along dim 0; 2-D
+    group-wise scales repeat over their group."""
+    s = np.asarray(scales, dtype=np.float64)
+    if s.ndim == 1:
+        return np.broadcast_to(s[:, None] if axis == 1 else s[None, :], shape)
+    if axis == 1:
+        return np.repeat(s, shape[1] // s.shape[1], axis=1)
+    return np.repeat(s, shape[0] // s.shape[0], axis=0)
+
+
+def rotation_rounding_band(t, scales, blk: int, axis: int) -> np.ndarray:
+    """Upper bound, in the units of the pre-rounding value t = v / s, on how far
+    the GPU's fp32 evaluation of t can lie from the oracle's fp64 one.
+
+    The b-point transform is log2(b) levels of additions, each partial sum
+    rounded once, so each output is off by at most log2(b) u sum_j |x_j| / sqrt(b)
+    (u = 2^-24, x the block's inputs; pairwise summation), and
+    sum_j |x_j| / sqrt(b) <= ||x||_2 = ||v_block||_2 (the normalised transform is
+    orthogonal).  The scale comes from the largest |v| of its group, computed the
+    same way, whose relative error is at most log2(b) u sqrt(b).  Bit-exact codes
+    cannot be asked for where t lies closer to a rounding midpoint than this:
+    the transform is evaluated in fp32 and its rounding may carry t across.  The
+    bound is small except where the block's outputs cancel to far below its
+    inputs (|v| much less than ||v_block||), e.g. next to outlier channels."""
+    t = np.asarray(t, dtype=np.float64)
+    se = _scale_per_element(scales, t.shape, axis)
+    v = t * se
+    rows, cols = t.shape
+    if axis == 1:
+        nrm = np.sqrt((v.reshape(rows, cols // blk, blk) ** 2).sum(axis=2))
+        nrm = np.repeat(nrm, blk, axis=1)
+    else:
+        nrm = np.sqrt((v.reshape(rows // blk, blk, cols) ** 2).sum(axis=1))
+        nrm = np.repeat(nrm, blk, axis=0)
+    lg = np.log2(blk)
+    u = 2.0 ** -24
+    with np.errstate(divide="ignore", invalid="ignore"):
+        band = lg * u * (np.where(se > 0, nrm / se, 0.0) + np.sqrt(blk) * np.abs(t))
+    return band
+
+
+def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype, blk=None, axis=None):
+    """Returns (#exempt elements, #exempt elements that differ).  With `blk` and
+    `axis` (1: blocks along the contiguous dim, 0: along dim 0) the exemption
+    also covers the fp32 transform's rounding bound (rotation_rounding_band)."""
     g = u8(gpu_codes)
     gs = gpu_scales.detach().cpu().numpy().astype(np.float64)
     os_ = np.asarray(ora_scales, dtype=np.float64)
@@ -28,22 +74,41 @@ def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype):
     assert np.all(gs[zero] == 0), "zero groups must give zero scales"
     rel = np.abs(gs[~zero] - os_[~zero]) / os_[~zero]
     assert rel.size == 0 or rel.max() <= SCALE_REL, f"scale rel err {rel.max():.3e}"
-    exempt = oracle.boundary_distance(ora_t, qtype) < BOUNDARY_REL
+    rel_d = oracle.boundary_distance(ora_t, qtype)
+    exempt = rel_d < BOUNDARY_REL
+    if blk is not None:
+        with np.errstate(invalid="ignore"):  # t = 0 has no midpoint (relative distance inf)
+            exempt |= rel_d * np.abs(ora_t) <= rotation_rounding_band(ora_t, ora_scales, blk, axis)
     diff = g != ora_codes
     bad = diff & ~exempt
     if bad.any():
         idx = np.argwhere(bad)[:5]
         details = [(tuple(i), int(g[tuple(i)]), int(ora_codes[tuple(i)]), float(ora_t[tuple(i)])) for i in idx]
         raise AssertionError(f"{int(bad.sum())} code mismatches outside the boundary band, e.g. {details}")
+    far = diff & exempt & ~_one_step_apart(g, np.asarray(ora_codes), qtype)
+    assert not far.any(), f"{int(far.sum())} exempt codes differ by more than one quantisation step"
     return int(exempt.sum()), int((diff & exempt).sum())
 
 
-def check_codes_stochastic(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, rand_bits, qtype, band=1e-4):
+def _one_step_apart(a, b, qtype) -> np.ndarray:
+    """Codes that are equal or neighbours on the quantisation grid."""
+    if qtype == oracle.INT8:
+        return np.abs(a.view(np.int8).astype(np.int16) - b.view(np.int8).astype(np.int16)) <= 1
+    da = oracle.e4m3_decode(a)
+    db = oracle.e4m3_decode(b)
+    m = np.maximum(np.abs(da), np.abs(db))
+    step = np.where(m <= 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(m, 2.0 ** -6))) - 3))
+    return np.abs(da - db) <= step
+
+
+def check_codes_stochastic(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, rand_bits, qtype, band=1e-4,
+                           blk=None, axis=None):
     """Stochastic rounding: codes must match the oracle's except where the
     decision is within `band` of flipping -- the random threshold u close to the
     oracle's fraction p = (t - lo) / (hi - lo), or t close to a grid point (p
-    near 0 or 1) -- since the GPU forms t in fp32 (about 1e-7 relative).
-    Returns (#exempt, #exempt that differ)."""
+    near 0 or 1) -- since the GPU forms t in fp32 (about 1e-7 relative).  With
+    `blk` and `axis` the band also covers the fp32 transform's rounding bound
+    (rotation_rounding_band) in units of p.  Returns (#exempt, #exempt that differ)."""
     g = u8(gpu_codes)
     gs = gpu_scales.detach().cpu().numpy().astype(np.float64)
     os_ = np.asarray(ora_scales, dtype=np.float64)
@@ -59,7 +124,11 @@ def check_codes_stochastic(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, 
         a = np.abs(t)
         quantum = np.where(a < 2.0**-6, 2.0**-9, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-300))) - 3))
         p = (a - np.floor(a / quantum) * quantum) / quantum
-    exempt = (np.abs(u - p) < band) | (p < band) | (p > 1 - band)
+    bp = np.full(t.shape, band)
+    if blk is not None:
+        q_unit = 1.0 if qtype == oracle.INT8 else quantum
+        bp = np.maximum(bp, rotation_rounding_band(t, ora_scales, blk, axis) / q_unit)
+    exempt = (np.abs(u - p) < bp) | (p < bp) | (p > 1 - bp)
     diff = g != ora_codes
     bad = diff & ~exempt
     if bad.any():

@@ -25,5 +25,5 @@ def test_bounded_wait_runs_out_and_is_reported():
     q, s = halo.halo_hadamard_quantize(x.to("cuda"), halo.HALO_AXIS_COLS, 128, halo.HALO_Q_INT8)
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x, 1, 128, halo.HALO_Q_INT8)
-    check_codes(q, s, codes, scales, t, halo.HALO_Q_INT8)
+    check_codes(q, s, codes, scales, t, halo.HALO_Q_INT8, blk=128, axis=1)
     assert halo.halo_device_error() == (halo.HALO_OK, 0)

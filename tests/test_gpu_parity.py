@@ -36,14 +36,18 @@ def _cuda(t):
 # ------------------------------------------------------------------ rotate + quantise
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
 @pytest.mark.parametrize("rows,cols,blk", [(300, 640, 128), (130, 512, 256), (1, 128, 128), (64, 256, 256),
-                                           (37, 11008, 128), (5, 28672, 128)])
+                                           (37, 11008, 128), (5, 28672, 128),
+                                           # rows per row group >= 3 (stage refills), codes in the consumed stage
+                                           (2000, 8192, 128), (600, 24576, 128),
+                                           # row groups of 4, 5 (code tiles) and 6 warps (codes in the stage)
+                                           (4, 16384, 128), (3, 20480, 128), (3, 24576, 128)])
 def test_rotq_rows_parity(qtype, rows, cols, blk):
     x = inputs.activations(rows, cols, seed=rows * 7 + cols, device="cpu")
     x[min(3, rows - 1)] = 0  # an all-zero row: scale 0, codes 0
     q, s = halo.halo_hadamard_quantize(_cuda(x), COLS, blk, qtype)
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x, 1, blk, qtype)
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=blk, axis=1)
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
@@ -55,7 +59,7 @@ def test_rotq_cols_parity(qtype, rows, cols):
     q, s = halo.halo_hadamard_quantize(_cuda(x), ROWS, 128, qtype)
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x, 0, 128, qtype)
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=128, axis=0)
 
 
 def test_rotq_rows_strided_input():
@@ -65,7 +69,7 @@ def test_rotq_rows_strided_input():
     q, s = halo.halo_hadamard_quantize(xd, COLS, 128, INT8)
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x.contiguous(), 1, 128, INT8)
-    check_codes(q, s, codes, scales, t, INT8)
+    check_codes(q, s, codes, scales, t, INT8, blk=128, axis=1)
 
 
 # ------------------------------------------------------------------------------ GEMM
@@ -144,8 +148,8 @@ def test_linear_fwd_tiny_config():
     torch.cuda.synchronize()
     cx, osx, tx = oracle_operand(x, 1, 256, INT8)
     cw, osw, tw = oracle_operand(w, 1, 256, INT8)
-    check_codes(qx, sx, cx, osx, tx, INT8)
-    check_codes(qw, sw, cw, osw, tw, INT8)
+    check_codes(qx, sx, cx, osx, tx, INT8, blk=256, axis=1)
+    check_codes(qw, sw, cw, osw, tw, INT8, blk=256, axis=1)
     ref = oracle.linear_fwd(x, w, 256, INT8)
     check_output(y, ref)
 
@@ -217,7 +221,8 @@ def test_full_rotate_quantize_16384x4096(qtype):
     rows = _sample(16384, 256, 1)
     xs = x[torch.from_numpy(rows).cuda()].cpu()
     codes, scales, t = oracle_operand(xs, 1, 128, qtype)
-    check_codes(q[torch.from_numpy(rows).cuda()], s[torch.from_numpy(rows).cuda()], codes, scales, t, qtype)
+    sel = torch.from_numpy(rows).cuda()
+    check_codes(q[sel], s[sel], codes, scales, t, qtype, blk=128, axis=1)
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
@@ -298,7 +303,7 @@ def test_random_sign_rotation_parity(qtype, axis, rows, cols, blk):
     torch.cuda.synchronize()
     v = oracle.rotate_signed(x, blk, 1 if axis == COLS else 0, s.numpy())
     codes, scales, t = oracle.quantize(v, axis=0 if axis == COLS else 1, qtype=qtype)
-    check_codes(q, sc, codes, scales, t, qtype)
+    check_codes(q, sc, codes, scales, t, qtype, blk=blk, axis=1 if axis == COLS else 0)
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
@@ -313,7 +318,8 @@ def test_stochastic_rounding_parity(qtype, axis, rows, cols, blk):
     codes, scales, t = oracle.quantize_stochastic(v, 0 if axis == COLS else 1, qtype, rb.numpy())
     from tests._parity import check_codes_stochastic
 
-    n_ex, n_diff = check_codes_stochastic(q, sc, codes, scales, t, rb.numpy(), qtype)
+    n_ex, n_diff = check_codes_stochastic(q, sc, codes, scales, t, rb.numpy(), qtype, blk=blk,
+                                          axis=1 if axis == COLS else 0)
     assert n_ex < 0.01 * x.numel()
 
 
@@ -329,7 +335,7 @@ def test_signs_and_stochastic_rounding_together_and_strided_random_bits():
     codes, scales, t = oracle.quantize_stochastic(v, 0, INT8, rb.contiguous().numpy())
     from tests._parity import check_codes_stochastic
 
-    check_codes_stochastic(q, sc, codes, scales, t, rb.contiguous().numpy(), INT8)
+    check_codes_stochastic(q, sc, codes, scales, t, rb.contiguous().numpy(), INT8, blk=128, axis=1)
 
 
 def test_random_sign_gemm_keeps_the_product():
@@ -361,7 +367,7 @@ def test_rotq_dual_parity(rows, cols, blk):
     torch.cuda.synchronize()
     for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
         codes, scales, t = oracle_operand(x, 1, blk, qt)
-        check_codes(q, s, codes, scales, t, qt)
+        check_codes(q, s, codes, scales, t, qt, blk=blk, axis=1)
         # byte for byte what the single-output call writes
         q1, s1 = halo.halo_hadamard_quantize(xd, COLS, blk, qt)
         torch.cuda.synchronize()
@@ -378,13 +384,14 @@ def test_rotq_dual_full_size_16384x4096():
     xs = x[rows].cpu()
     for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
         codes, scales, t = oracle_operand(xs, 1, 128, qt)
-        check_codes(q[rows], s[rows], codes, scales, t, qt)
+        check_codes(q[rows], s[rows], codes, scales, t, qt, blk=128, axis=1)
 
 
 # ------------------------------------------------------------ zero padding (ragged lengths)
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
 @pytest.mark.parametrize("rows,cols,blk", [(37, 1000, 128), (5, 296, 256), (9, 72, 128), (3, 200, 256),
-                                           (4, 32760, 128), (6, 384, 256)])
+                                           (4, 32760, 128), (6, 384, 256), (3, 24504, 128), (300, 20000, 128),
+                                           (2000, 8000, 128)])
 def test_rotq_rows_padded_parity(qtype, rows, cols, blk):
     """Row length not a multiple of blk: the partial chunk arrives by its own
     TMA box (zeros past the row), whole padding chunks are zeros; the codes
@@ -394,7 +401,7 @@ def test_rotq_rows_padded_parity(qtype, rows, cols, blk):
     torch.cuda.synchronize()
     assert tuple(q.shape) == (rows, halo.padded_length(cols, blk))
     codes, scales, t = oracle_operand(x, 1, blk, qtype)
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=blk, axis=1)
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
@@ -407,7 +414,7 @@ def test_rotq_cols_padded_parity(qtype, rows, cols):
     torch.cuda.synchronize()
     assert tuple(q.shape) == (halo.padded_length(rows, 128), cols)
     codes, scales, t = oracle_operand(x, 0, 128, qtype)
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=128, axis=0)
 
 
 def test_rotq_dual_padded_parity():
@@ -416,7 +423,7 @@ def test_rotq_dual_padded_parity():
     torch.cuda.synchronize()
     for q, s, qt in ((q8, s8, INT8), (qf, sf, E4M3)):
         codes, scales, t = oracle_operand(x, 1, 128, qt)
-        check_codes(q, s, codes, scales, t, qt)
+        check_codes(q, s, codes, scales, t, qt, blk=128, axis=1)
 
 
 @pytest.mark.parametrize("axis,rows,cols", [(COLS, 37, 1000), (ROWS, 1000, 48)])
@@ -434,7 +441,7 @@ def test_padded_variants_parity(axis, rows, cols):
     along = 1 if axis == COLS else 0
     v = oracle.rotate_signed(x, 128, along, s.numpy()[:n])
     codes, scales, t = oracle.quantize_stochastic(v, 0 if along == 1 else 1, INT8, rb.numpy().view(np.uint16))
-    check_codes_stochastic(q, sc, codes, scales, t, rb.numpy().view(np.uint16), INT8)
+    check_codes_stochastic(q, sc, codes, scales, t, rb.numpy().view(np.uint16), INT8, blk=128, axis=along)
 
 
 @pytest.mark.parametrize("blk", [128, 256])
@@ -465,7 +472,8 @@ def test_linear_bwd_padded_n_and_m():
 # -------------------------------------------------------------- group-wise scales
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
 @pytest.mark.parametrize("rows,cols,blk,group", [(300, 640, 128, 64), (300, 640, 128, 128), (130, 512, 256, 64),
-                                                 (5, 1000, 128, 64), (3, 28672, 128, 128)])
+                                                 (5, 1000, 128, 64), (3, 28672, 128, 128), (3, 24576, 128, 64),
+                                                 (300, 28672, 128, 128), (2000, 8192, 128, 64)])
 def test_rotq_rows_grouped_parity(qtype, rows, cols, blk, group):
     x = inputs.activations(rows, cols, seed=rows + 2 * cols + group, device="cpu")
     x[min(1, rows - 1), :64] = 0  # an all-zero group
@@ -473,7 +481,7 @@ def test_rotq_rows_grouped_parity(qtype, rows, cols, blk, group):
     torch.cuda.synchronize()
     codes, scales, t = oracle.quantize_grouped(oracle.rotate(x, blk, 1), 1, group, qtype)
     assert tuple(s.shape) == scales.shape
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=blk, axis=1)
 
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
@@ -486,7 +494,7 @@ def test_rotq_cols_grouped_parity(qtype, rows, cols, group):
     torch.cuda.synchronize()
     codes, scales, t = oracle.quantize_grouped(oracle.rotate(x, 128, 0), 0, group, qtype)
     assert tuple(s.shape) == scales.shape
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=128, axis=0)
 
 
 def _group_scales(outer, ngroups, seed):
@@ -579,4 +587,4 @@ def test_rotq_rows_longest_row(qtype):
     q, s = halo.halo_hadamard_quantize(_cuda(x), COLS, 128, qtype)
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x, 1, 128, qtype)
-    check_codes(q, s, codes, scales, t, qtype)
+    check_codes(q, s, codes, scales, t, qtype, blk=128, axis=1)
