@@ -195,10 +195,6 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t phase) {
   uint32_t ok;
   asm volatile(
