@@ -155,6 +155,8 @@ halo_status_t device_setup(int* dev_out) {
     HALO_CUDA(set_smem_attr(rotq_cols_grouped_kernel<1>, optin));
     HALO_CUDA(set_smem_attr(qgemm_grouped_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_grouped_kernel<1>, optin));
+    HALO_CUDA(set_smem_attr(rotq_rows_pair_kernel<0>, optin));
+    HALO_CUDA(set_smem_attr(rotq_rows_pair_kernel<1>, optin));
     for (int pad = 0; pad < 2; ++pad) {
       for (int qt = 0; qt < 2; ++qt) {
         HALO_CUDA(set_smem_attr(rows_kernel(128, qt, false, pad, true), optin));
@@ -268,6 +270,57 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 int64_t pad_to(int64_t n, int64_t b) { return (n + b - 1) / b * b; }
 
 // ------------------------------------------------------------------------ rotq launches
+// Rows of 193..256 whole 128-element chunks (whole blocks of 128, one output):
+// each row split over a cluster of two CTAs of 4 warps (rotq_rows_pair_kernel).
+bool rows_pair_applies(int64_t cols, int blk, int qtype, bool ext, int group) {
+  if (blk != 128 || ext || group != 0 || (qtype != HALO_Q_INT8 && qtype != HALO_Q_E4M3) || cols % 128 != 0)
+    return false;
+  const int64_t nb = cols / 128;
+  return nb > 192 && nb <= 256 && nb % 2 == 0;
+}
+
+halo_status_t launch_rotq_rows_pair(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
+                                    int64_t ld_q, float* scales, cudaStream_t stream, int dev) {
+  const int nb = static_cast<int>(cols / 128);
+  const int h = nb / 2;
+  CUtensorMap tm_x, tm_q;
+  {
+    // [rows][nb][128] with a 136-element inner box: the 8 elements past each
+    // chunk are out of range and arrive as zeros (a 272-byte slot per thread).
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[3] = {kRowsInSlot / 2, static_cast<cuuint32_t>(h), 1};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(nb), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[3] = {kRowsOutSlot, static_cast<cuuint32_t>(h), 1};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  RotqRowsPairParams p;
+  p.scales = scales;
+  p.rows = rows;
+  p.h = h;
+  p.qmax = qtype == HALO_Q_E4M3 ? 448.f : 127.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  auto kern = qtype == HALO_Q_INT8 ? rotq_rows_pair_kernel<0> : rotq_rows_pair_kernel<1>;
+  // Persistent: as many two-CTA clusters as fit at once, each looping over rows.
+  Launch L(dim3(2), dim3(128), 2 * kRowsPairStageBytes + 128, stream, 2);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &L.cfg) != cudaSuccess || max_clusters < 1) {
+    (void)cudaGetLastError();
+    max_clusters = g_dev[dev].sm_count;
+  }
+  L.cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<int64_t>(rows, max_clusters)));
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
 // qtype kQtDual: q / ld_q / scales take the INT8 output, q2 / ld_q2 / scales2
 // the E4M3 one (unused otherwise).
 halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int blk, int qtype,
@@ -275,6 +328,8 @@ halo_status_t launch_rotq_rows(const void* x, int64_t rows, int64_t cols, int64_
                                cudaStream_t stream, int dev, void* q2 = nullptr, int64_t ld_q2 = 0,
                                float* scales2 = nullptr, int group = 0) {
   const bool dual = qtype == kQtDual;
+  if (!dual && rows_pair_applies(cols, blk, qtype, ext, group))
+    return launch_rotq_rows_pair(x, rows, cols, ld_x, qtype, q, ld_q, scales, stream, dev);
   // A row of `cols` elements is zero-padded to whole blocks: nb 128-element
   // chunks, of which nbt are whole in the input and one more (tail > 0
   // elements) is partial; chunks past that are all zero.

@@ -5,6 +5,8 @@
 //   rotq_rows_kernel        rotate along the contiguous dimension (blocks of
 //                           128 or 256 consecutive elements of a row), one
 //                           scale per row (or per group of 64 / 128 elements).
+//   rotq_rows_pair_kernel   the same for rows of 193..256 whole 128-element
+//                           blocks, each row split over a two-CTA cluster.
 //   rotq_cols_1pass_kernel  rotate along dimension 0 (blocks of 128
 //   rotq_cols_kernel        consecutive rows of a column), one scale per
 //                           column: a single pass for up to 8192 rows, two
@@ -518,6 +520,155 @@ __global__ void __launch_bounds__(BLK == 128 && EXT == 0 && QT != kQtDual ? 384 
     }
   }
   if (leader) bulk_wait<0>();
+}
+
+// ------------------------------------------------------------------------------------------
+// rotq_rows_pair: rows of 193..256 whole 128-element chunks (e.g. 28672
+// elements), each split over a cluster of two CTAs of 4 warps: rank r owns
+// chunks [r h, r h + h), h = nb / 2 <= 128, one thread per chunk.  One CTA per
+// row would need 7-8 warps and two ~61 KB input stages, i.e. one CTA (7-8
+// warps) per SM; the halves fit three CTAs (12 warps) per SM.  Each CTA's
+// half-row maximum goes to the partner's slot with one 16-byte st.async that
+// completes bytes on the partner's mbarrier; two slot buffers alternate over
+// rows (the partner writes row k+2's slot only after it has this CTA's row k+1
+// maximum, which is sent after this CTA has read row k's slot).  Codes are
+// written into the consumed input stage, which is refilled with the next row
+// once their store has read them.
+// ------------------------------------------------------------------------------------------
+struct RotqRowsPairParams {
+  float* scales;
+  int64_t rows;
+  int h;             // chunks per CTA (nb / 2)
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(128))
+};
+
+enum : unsigned int { kSiteRotqPairLoad = 0x105, kSiteRotqPairReduce = 0x106 };
+
+constexpr uint32_t kRowsPairStageBytes = 128 * kRowsInSlot;  // one stage: up to 128 chunk slots
+
+template <int QT>
+__global__ void __launch_bounds__(128, 3)
+    rotq_rows_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                          RotqRowsPairParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t full_bar[2];                 // input stage loaded
+  __shared__ uint64_t red_bar[2];                  // partner's maximum received, per row parity
+  __shared__ uint32_t s_wmax[2][4];                // per-warp maxima, per row parity
+  __shared__ __align__(16) uint32_t s_slot[2][4];  // the partner's half-row maximum (element 0)
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t peer = crank ^ 1u;
+  const int chunk = threadIdx.x;  // this thread's chunk within the CTA's half row
+  const bool is_active = chunk < p.h;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&full_bar[0], 1);
+    mbar_init(&full_bar[1], 1);
+    mbar_init(&red_bar[0], 1);
+    mbar_init(&red_bar[1], 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_q);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&red_bar[0], 16);  // armed for rows 0 and 1
+    mbar_arrive_expect_tx(&red_bar[1], 16);
+  }
+  cluster_arrive();  // the partner is running and initialised before the first remote store
+  cluster_wait();
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const int64_t cid = blockIdx.x / 2;  // this cluster: rows cid, cid + ncl, ...
+  const int64_t ncl = gridDim.x / 2;
+  const int64_t nmine = cid < p.rows ? (p.rows - cid + ncl - 1) / ncl : 0;
+
+  auto issue = [&](int64_t it) {
+    const int st = static_cast<int>(it & 1);
+    mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(p.h) * kRowsInSlot);
+    tma_load_3d(smem + st * kRowsPairStageBytes, &tm_x, &full_bar[st], 0, static_cast<int32_t>(crank) * p.h,
+                static_cast<int32_t>(cid + it * ncl));
+  };
+  if (threadIdx.x == 0) {
+    if (nmine > 0) issue(0);
+    if (nmine > 1) issue(1);
+  }
+
+  bool dead = false;  // a wait ran out: stop waiting and loading, keep every barrier and send every maximum
+  for (int64_t it = 0; it < nmine; ++it) {
+    const int st = static_cast<int>(it & 1);
+    const uint32_t ph = static_cast<uint32_t>((it >> 1) & 1);
+    const int64_t row = cid + it * ncl;
+    uint8_t* stage = smem + st * kRowsPairStageBytes;
+    if (!dead) dead = !mbar_wait(&full_bar[st], ph, kSiteRotqPairLoad);
+    float2 v[64];
+    if (is_active && !dead) {
+      const uint4* src = reinterpret_cast<const uint4*>(stage + chunk * kRowsInSlot);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const uint4 raw = src[k];
+        v[4 * k + 0] = bf16x2_to_f2(raw.x);
+        v[4 * k + 1] = bf16x2_to_f2(raw.y);
+        v[4 * k + 2] = bf16x2_to_f2(raw.z);
+        v[4 * k + 3] = bf16x2_to_f2(raw.w);
+      }
+      fwht128_pairs(v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
+    }
+    __syncthreads();  // stage `st` fully read
+    if (threadIdx.x == 0 && !dead && it >= 1 && it + 1 < nmine) {
+      // The other stage holds the previous row's codes: once their store has
+      // read them, it takes the next row.
+      bulk_wait_read<0>();
+      issue(it + 1);
+    }
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(absmax128(v)));
+    if (lane == 0) s_wmax[st][warp] = wmax;
+    __syncthreads();
+    const uint32_t cmax = max(max(s_wmax[st][0], s_wmax[st][1]), max(s_wmax[st][2], s_wmax[st][3]));
+    if (threadIdx.x == 0)
+      st_async_v4(map_to_rank(&s_slot[st][0], peer), make_uint4(cmax, 0u, 0u, 0u), map_to_rank(&red_bar[st], peer));
+    if (!dead) dead = !mbar_wait_cluster(&red_bar[st], ph, kSiteRotqPairReduce);
+    const uint32_t pmax = s_slot[st][0];
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&red_bar[st], 16);  // re-armed for row it + 2
+    const float row_amax = __uint_as_float(max(cmax, pmax));
+    const float r = row_amax > 0.f ? __fdiv_rn(p.qmax, row_amax) : 0.f;
+    if (crank == 0 && threadIdx.x == 0) p.scales[row] = row_amax * p.scale_mult;
+    if (is_active) {
+      uint4* dst = reinterpret_cast<uint4*>(stage + chunk * kRowsOutSlot);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 a = v[8 * k + 2 * j];
+          const float2 b = v[8 * k + 2 * j + 1];
+          if (QT == 0)
+            w[j] = pack4_int8(q_int8_bits(a.x, r), q_int8_bits(a.y, r), q_int8_bits(b.x, r), q_int8_bits(b.y, r));
+          else
+            w[j] = e4m3x2_bits(a.x * r, a.y * r) | (e4m3x2_bits(b.x * r, b.y * r) << 16);
+        }
+        dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tma_store_3d(&tm_q, stage, 0, static_cast<int32_t>(crank) * p.h, static_cast<int32_t>(row));
+      bulk_commit();
+    }
+  }
+  if (threadIdx.x == 0) bulk_wait<0>();
+  __syncthreads();
+  cluster_arrive();  // no CTA leaves while its partner could still store into its shared memory
+  cluster_wait();
 }
 
 constexpr int kColsStrip = 32;

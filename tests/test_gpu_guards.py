@@ -56,7 +56,9 @@ def _check_vec(buf, n):
                                                 (halo.HALO_AXIS_COLS, 37, 640, 256),
                                                 (halo.HALO_AXIS_ROWS, 1000, 48, 128),
                                                 (halo.HALO_AXIS_ROWS, 8320, 32, 128),
-                                                (halo.HALO_AXIS_ROWS, 4096, 208, 128)])
+                                                (halo.HALO_AXIS_ROWS, 4096, 208, 128),
+                                                (halo.HALO_AXIS_COLS, 700, 8192, 128),
+                                                (halo.HALO_AXIS_COLS, 500, 28672, 128)])
 def test_rotate_quantize_writes_only_its_outputs(qtype, axis, rows, cols, blk):
     x = inputs.activations(rows, cols, seed=rows + cols, device="cuda")
     qr, qc = halo.codes_shape(rows, cols, axis, blk)

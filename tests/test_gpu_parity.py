@@ -39,6 +39,8 @@ def _cuda(t):
                                            (37, 11008, 128), (5, 28672, 128),
                                            # rows per row group >= 3 (stage refills), codes in the consumed stage
                                            (2000, 8192, 128), (600, 24576, 128),
+                                           # rows split over two-CTA clusters, >= 3 rows per cluster
+                                           (700, 28672, 128), (2, 25600, 128),
                                            # row groups of 4, 5 (code tiles) and 6 warps (codes in the stage)
                                            (4, 16384, 128), (3, 20480, 128), (3, 24576, 128)])
 def test_rotq_rows_parity(qtype, rows, cols, blk):
