@@ -80,6 +80,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigne
   }
 }
 
+// Before a CTA returns: wait, bounded, until the last TMA load issued into
+// each stage of a ring has landed, so that no copy still writes into this
+// CTA's shared memory after it exits.  In a normal run every load has been
+// consumed already and this returns at once; it matters after a wait ran out
+// and the kernel stopped consuming its ring.  Bit s of `issued`: stage s
+// received a load; bit s of `parity`: the phase parity of the last one.
+constexpr unsigned long long kDrainLimitNs = 200000000ull;  // 200 ms per stage
+
+__device__ __forceinline__ void drain_loads(uint64_t* bars, int nstages, uint32_t issued, uint32_t parity,
+                                            unsigned int site) {
+  for (int s = 0; s < nstages; ++s)
+    if ((issued >> s) & 1u) (void)mbar_wait(&bars[s], (parity >> s) & 1u, site, kDrainLimitNs);
+}
+
+// Records a load into stage s with phase parity `par` for drain_loads().
+__device__ __forceinline__ void note_load(uint32_t& issued, uint32_t& parity, int s, uint32_t par) {
+  issued |= 1u << s;
+  parity = (parity & ~(1u << s)) | ((par & 1u) << s);
+}
+
 // ------------------------------------------------- programmatic dependent launch
 // Wait until the preceding kernel in the stream has completed and its memory is
 // visible (returns at once when the launch has no programmatic dependency).

@@ -31,6 +31,7 @@ enum : unsigned int {
   kSiteGemmMma = 0x302,
   kSiteGemmMmaAcc = 0x303,
   kSiteGemmEpilogue = 0x304,
+  kSiteGemmDrain = 0x305,
 };
 
 constexpr int kGemmBM = 128;
@@ -114,11 +115,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain below
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int tm, tn;
         gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, kSiteGemmProducer)) { ok = false; break; }
+          note_load(ld_issued, ld_par, stage, phase);
           mbar_arrive_expect_tx(&full[stage], kGemmABytes + kGemmBBytes);
           uint8_t* a_dst = sA + stage * kGemmABytes;
           uint8_t* b_dst = sB + stage * kGemmBBytes;
@@ -135,6 +138,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
         }
       }
+      drain_loads(full, kGemmStages, ld_issued, ld_par, kSiteGemmDrain);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -279,6 +283,7 @@ enum : unsigned int {
   kSitePairMma = 0x312,
   kSitePairMmaAcc = 0x313,
   kSitePairEpilogue = 0x314,
+  kSitePairDrain = 0x315,
 };
 
 template <int QT>
@@ -334,6 +339,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain below
       for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
         int tm, tn;
         gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
@@ -341,6 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int b_row = tn * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, kSitePairProducer)) { ok = false; break; }
+          note_load(ld_issued, ld_par, stage, phase);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
           const uint32_t bar = map_to_rank(&full[stage], 0);
           uint8_t* a_dst = sA + stage * kPairABytes;
@@ -356,6 +363,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
         }
       }
+      // Both CTAs' loads complete bytes on the leader's barriers: the leader
+      // drains them; the other CTA stays until the final cluster barrier.
+      if (leader) drain_loads(full, kPairStages, ld_issued, ld_par, kSitePairDrain);
     }
     __syncwarp();
   } else if (warp == 1) {

@@ -35,10 +35,11 @@
 namespace halo {
 
 enum : unsigned int {
-  kSiteGgProducer = 0x311,
-  kSiteGgMma = 0x312,
-  kSiteGgPartial = 0x313,
-  kSiteGgPromote = 0x314,
+  kSiteGgProducer = 0x321,
+  kSiteGgMma = 0x322,
+  kSiteGgPartial = 0x323,
+  kSiteGgPromote = 0x324,
+  kSiteGgDrain = 0x325,
 };
 
 constexpr int kGgBM = 128;
@@ -123,11 +124,13 @@ __global__ void __launch_bounds__(kGgThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain below
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int tm, tn;
         gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, kSiteGgProducer)) { ok = false; break; }
+          note_load(ld_issued, ld_par, stage, phase);
           mbar_arrive_expect_tx(&full[stage], kGgABytes + kGgBBytes);
           uint8_t* a_dst = sA + stage * kGgABytes;
           uint8_t* b_dst = sB + stage * kGgBBytes;
@@ -142,6 +145,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
           if (++stage == kGgStages) { stage = 0; phase ^= 1u; }
         }
       }
+      drain_loads(full, kGgStages, ld_issued, ld_par, kSiteGgDrain);
     }
     __syncwarp();
   } else if (warp == 1) {

@@ -40,7 +40,9 @@ namespace halo {
 
 enum : unsigned int {
   kSiteRotqRowsLoad = 0x101,
+  kSiteRotqRowsDrain = 0x102,
   kSiteRotqColsLoad = 0x201,
+  kSiteRotqColsDrain = 0x208,
 };
 
 // Per-thread slot sizes in shared memory for rotq_rows: 128 bf16 (256 B) plus
@@ -310,10 +312,12 @@ __global__ void __launch_bounds__(BLK == 128 && EXT == 0 && QT != kQtDual ? 384 
   const int64_t step = static_cast<int64_t>(gridDim.x) * p.groups;
   const int64_t nmine = first < p.rows ? (p.rows - first + step - 1) / step : 0;
 
+  uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain at the end
   auto issue = [&](int64_t it) {
     const int st = static_cast<int>(it & 1);
     const int32_t row = static_cast<int32_t>(first + it * step);
     uint8_t* dst = g_in + st * rows_group_in_bytes(gw, PAD);
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(it >> 1));
     mbar_arrive_expect_tx(&full_bar[grp][st], in_bytes);
     if (!PAD || p.nbt > 0) tma_load_3d(dst, &tm_x, &full_bar[grp][st], 0, 0, row);
     // Partial last chunk: elements past the row's end are out of the 2-D
@@ -519,7 +523,10 @@ __global__ void __launch_bounds__(BLK == 128 && EXT == 0 && QT != kQtDual ? 384 
       bulk_commit();  // one group for both stores: the wait above covers both tiles
     }
   }
-  if (leader) bulk_wait<0>();
+  if (leader) {
+    drain_loads(full_bar[grp], 2, ld_issued, ld_par, kSiteRotqRowsDrain);
+    bulk_wait<0>();
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -543,7 +550,7 @@ struct RotqRowsPairParams {
   float scale_mult;  // 1 / (qmax * sqrt(128))
 };
 
-enum : unsigned int { kSiteRotqPairLoad = 0x105, kSiteRotqPairReduce = 0x106 };
+enum : unsigned int { kSiteRotqPairLoad = 0x105, kSiteRotqPairReduce = 0x106, kSiteRotqPairDrain = 0x107 };
 
 constexpr uint32_t kRowsPairStageBytes = 128 * kRowsInSlot;  // one stage: up to 128 chunk slots
 
@@ -588,8 +595,10 @@ __global__ void __launch_bounds__(128, 3)
   const int64_t ncl = gridDim.x / 2;
   const int64_t nmine = cid < p.rows ? (p.rows - cid + ncl - 1) / ncl : 0;
 
+  uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain at the end
   auto issue = [&](int64_t it) {
     const int st = static_cast<int>(it & 1);
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(it >> 1));
     mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(p.h) * kRowsInSlot);
     tma_load_3d(smem + st * kRowsPairStageBytes, &tm_x, &full_bar[st], 0, static_cast<int32_t>(crank) * p.h,
                 static_cast<int32_t>(cid + it * ncl));
@@ -665,7 +674,10 @@ __global__ void __launch_bounds__(128, 3)
       bulk_commit();
     }
   }
-  if (threadIdx.x == 0) bulk_wait<0>();
+  if (threadIdx.x == 0) {
+    drain_loads(full_bar, 2, ld_issued, ld_par, kSiteRotqPairDrain);
+    bulk_wait<0>();
+  }
   __syncthreads();
   cluster_arrive();  // no CTA leaves while its partner could still store into its shared memory
   cluster_wait();
@@ -810,9 +822,11 @@ __global__ void __launch_bounds__(128, EXT ? 2 : 3)
   // blocks read last in pass 1 are the likeliest still to be in L2.
   const int nseq = 2 * nmine;
 
+  uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain at the end
   auto issue = [&](int j) {
     const int b = first + step * (j < nmine ? j : 2 * nmine - 1 - j);
     const int s = j % kColsStages;
+    note_load(ld_issued, ld_par, s, static_cast<uint32_t>(j / kColsStages));
     mbar_arrive_expect_tx(&bars[warp][s], kColsInBytes);
     tma_load_2d(s_in + s * kColsInBytes, &tm_x, &bars[warp][s], c0, b * 128);
   };
@@ -911,7 +925,10 @@ __global__ void __launch_bounds__(128, EXT ? 2 : 3)
       bulk_commit();
     }
   }
-  if (lane == 0) bulk_wait<0>();
+  if (lane == 0) {
+    drain_loads(bars[warp], kColsStages, ld_issued, ld_par, kSiteRotqColsDrain);
+    bulk_wait<0>();
+  }
   cluster_wait();  // every CTA of the cluster is done reading this CTA's s_part
 }
 
@@ -945,7 +962,7 @@ struct RotqCols1Params {
   RotqExtras ex;     // EXT = 1 only
 };
 
-enum : unsigned int { kSiteRotqCols1Load = 0x202, kSiteRotqCols1Reduce = 0x203 };
+enum : unsigned int { kSiteRotqCols1Load = 0x202, kSiteRotqCols1Reduce = 0x203, kSiteRotqCols1Drain = 0x205 };
 
 template <int QT, int NW, int EXT>
 __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
@@ -993,8 +1010,10 @@ __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
   const int step = gridDim.y;
   const int nmine = first < p.strips ? (p.strips - first + step - 1) / step : 0;
 
+  uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain at the end
   auto issue = [&](int k) {
     const int st = k & 1;
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(k >> 1));
     mbar_arrive_expect_tx(&bars[warp][st], kColsInBytes);
     tma_load_2d(s_in + st * kColsInBytes, &tm_x, &bars[warp][st], (first + k * step) * kColsStrip, blk * 128);
   };
@@ -1076,7 +1095,10 @@ __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
       bulk_commit();
     }
   }
-  if (lane == 0) bulk_wait<0>();
+  if (lane == 0) {
+    drain_loads(bars[warp], 2, ld_issued, ld_par, kSiteRotqCols1Drain);
+    bulk_wait<0>();
+  }
   __syncthreads();
   cluster_arrive();  // no CTA leaves while a peer could still store into its shared memory
   cluster_wait();
@@ -1101,7 +1123,7 @@ struct RotqColsGrParams {
   float scale_mult;  // 1 / (qmax * sqrt(128))
 };
 
-enum : unsigned int { kSiteRotqColsGrLoad = 0x204 };
+enum : unsigned int { kSiteRotqColsGrLoad = 0x204, kSiteRotqColsGrDrain = 0x206 };
 
 // Column-wise max |v| over 32 float2 (x and y are two columns), as trees.
 __device__ __forceinline__ float2 absmax32_cols(const float2* v) {
@@ -1150,10 +1172,12 @@ __global__ void __launch_bounds__(128, 3)
   const int64_t nw = static_cast<int64_t>(gridDim.x) * 4;
   const int64_t nmine = wid < items ? (items - wid + nw - 1) / nw : 0;
 
+  uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain at the end
   auto issue = [&](int64_t k) {
     const int64_t it = wid + k * nw;
     const int b = static_cast<int>(it / p.strips), sidx = static_cast<int>(it % p.strips);
     const int st = static_cast<int>(k & 1);
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(k >> 1));
     mbar_arrive_expect_tx(&bars[warp][st], kColsInBytes);
     tma_load_2d(s_in + st * kColsInBytes, &tm_x, &bars[warp][st], sidx * kColsStrip, b * 128);
   };
@@ -1226,7 +1250,10 @@ __global__ void __launch_bounds__(128, 3)
       bulk_commit();
     }
   }
-  if (lane == 0) bulk_wait<0>();
+  if (lane == 0) {
+    drain_loads(bars[warp], 2, ld_issued, ld_par, kSiteRotqColsGrDrain);
+    bulk_wait<0>();
+  }
 }
 
 }  // namespace halo
