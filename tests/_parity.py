@@ -1,5 +1,7 @@
 """Comparison helpers shared by the GPU parity tests (no method arithmetic here:
 the expected values always come from the oracle)."""
+import os
+
 import numpy as np
 import torch
 
@@ -14,6 +16,40 @@ BOUNDARY_REL = 1e-6
 SCALE_REL = 1e-6
 # Final fp32 / bf16 outputs: max |Y - Y_ref| / max |Y_ref|.
 OUT_REL = 1e-3
+# Ceilings on the share of an operand's codes that the band may exempt from
+# bit-exactness, so that a widened band cannot hide a systematic mismatch.
+# The exempt set depends on the oracle's values alone (fixed seeds), so these
+# checks cannot flake.  Round to nearest: 0.2% for 128-blocks, 0.4% for
+# 256-blocks (the fp32 transform's bound grows with the block); the test inputs
+# measure at most 0.16% and 0.36%, and 0.003%-0.08% on the large outlier
+# operands.  Stochastic rounding also exempts a decision within 1e-4 of
+# flipping (about 0.04% of codes) and every group's maximum (t = +-qmax lies on
+# the grid): 1%, against at most 0.45% measured.
+EXEMPT_MAX_FRAC_RNE_128 = 2e-3
+EXEMPT_MAX_FRAC_STOCHASTIC = 1e-2
+
+
+def rne_exempt_ceiling(blk) -> float:
+    return EXEMPT_MAX_FRAC_RNE_128 * (blk if blk else 128) / 128
+
+# One record per code comparison, printed at the end of the test session
+# (tests/conftest.py): which test, the shape and type, how many codes, how many
+# the 1e-6 relative term exempts, how many only the fp32 transform's bound
+# exempts, and how many exempt codes actually differ.
+EXEMPT_LOG = []
+
+
+def _record(kind, shape, qtype, n, by_rel, by_band, differ, ceiling):
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    EXEMPT_LOG.append({"test": test, "kind": kind, "shape": tuple(int(d) for d in shape),
+                       "qtype": "int8" if qtype == oracle.INT8 else "e4m3", "codes": int(n),
+                       "exempt_rel": int(by_rel), "exempt_band_only": int(by_band), "differ": int(differ),
+                       "ceiling": ceiling})
+    frac = (by_rel + by_band) / max(n, 1)
+    assert frac <= ceiling, (
+        f"the band exempts {by_rel + by_band} of {n} codes ({100 * frac:.3f}%, "
+        f"{by_rel} by the fixed relative term, {by_band} by the fp32 transform bound only), "
+        f"above the {100 * ceiling:.1f}% ceiling")
 
 
 def u8(t: torch.Tensor) -> np.ndarray:
@@ -66,7 +102,9 @@ def rotation_rounding_band(t, scales, blk: int, axis: int) -> np.ndarray:
 def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype, blk=None, axis=None):
     """Returns (#exempt elements, #exempt elements that differ).  With `blk` and
     `axis` (1: blocks along the contiguous dim, 0: along dim 0) the exemption
-    also covers the fp32 transform's rounding bound (rotation_rounding_band)."""
+    also covers the fp32 transform's rounding bound (rotation_rounding_band).
+    The counts, split by the term that exempts each code, are recorded in
+    EXEMPT_LOG, and the exempt share must stay within EXEMPT_MAX_FRAC."""
     g = u8(gpu_codes)
     gs = gpu_scales.detach().cpu().numpy().astype(np.float64)
     os_ = np.asarray(ora_scales, dtype=np.float64)
@@ -75,11 +113,14 @@ def check_codes(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, qtype, blk=
     rel = np.abs(gs[~zero] - os_[~zero]) / os_[~zero]
     assert rel.size == 0 or rel.max() <= SCALE_REL, f"scale rel err {rel.max():.3e}"
     rel_d = oracle.boundary_distance(ora_t, qtype)
-    exempt = rel_d < BOUNDARY_REL
+    by_rel = rel_d < BOUNDARY_REL
+    exempt = by_rel.copy()
     if blk is not None:
         with np.errstate(invalid="ignore"):  # t = 0 has no midpoint (relative distance inf)
             exempt |= rel_d * np.abs(ora_t) <= rotation_rounding_band(ora_t, ora_scales, blk, axis)
     diff = g != ora_codes
+    _record("rne", g.shape, qtype, g.size, by_rel.sum(), (exempt & ~by_rel).sum(), (diff & exempt).sum(),
+            rne_exempt_ceiling(blk))
     bad = diff & ~exempt
     if bad.any():
         idx = np.argwhere(bad)[:5]
@@ -125,11 +166,18 @@ def check_codes_stochastic(gpu_codes, gpu_scales, ora_codes, ora_scales, ora_t, 
         quantum = np.where(a < 2.0**-6, 2.0**-9, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-300))) - 3))
         p = (a - np.floor(a / quantum) * quantum) / quantum
     bp = np.full(t.shape, band)
+    bp_rel = bp
     if blk is not None:
         q_unit = 1.0 if qtype == oracle.INT8 else quantum
         bp = np.maximum(bp, rotation_rounding_band(t, ora_scales, blk, axis) / q_unit)
-    exempt = (np.abs(u - p) < bp) | (p < bp) | (p > 1 - bp)
+    # t = 0 exactly (an all-zero group, or zero padding meeting zeros) is code 0
+    # on both sides: nothing to exempt there.
+    nz = t != 0
+    by_rel = nz & ((np.abs(u - p) < bp_rel) | (p < bp_rel) | (p > 1 - bp_rel))
+    exempt = nz & ((np.abs(u - p) < bp) | (p < bp) | (p > 1 - bp))
     diff = g != ora_codes
+    _record("stochastic", g.shape, qtype, g.size, by_rel.sum(), (exempt & ~by_rel).sum(), (diff & exempt).sum(),
+            EXEMPT_MAX_FRAC_STOCHASTIC)
     bad = diff & ~exempt
     if bad.any():
         idx = np.argwhere(bad)[:5]

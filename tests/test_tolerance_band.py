@@ -70,3 +70,31 @@ def test_band_covers_the_crossing_seen_on_the_gpu():
     band = rotation_rounding_band(t64, scales, 128, 1)
     assert abs(t64[0, j] - mid) <= band[0, j]
     assert abs(t64[0, j] - mid) > 1e-6 * abs(t64[0, j])  # outside the relative band alone
+
+
+def test_exemption_counts_are_recorded_and_bounded(monkeypatch):
+    """check_codes records how many codes each term of the band exempts, and
+    fails when the exempt share passes its ceiling.  Here the oracle's own
+    codes stand in for the GPU's (nothing differs); widening the fixed relative
+    term to 0.05 exempts ~10% of the codes and must trip the ceiling."""
+    import torch
+
+    from tests import _parity
+
+    x = inputs.activations(64, 1024, seed=5, device="cpu")
+    for qt in (oracle.INT8, oracle.E4M3):
+        codes, scales, t = _parity.oracle_operand(x, 1, 128, qt)
+        gpu_codes = torch.from_numpy(np.ascontiguousarray(codes))
+        gpu_scales = torch.from_numpy(np.asarray(scales, dtype=np.float32))
+        before = len(_parity.EXEMPT_LOG)
+        n_ex, n_diff = _parity.check_codes(gpu_codes, gpu_scales, codes, scales, t, qt, blk=128, axis=1)
+        rec = _parity.EXEMPT_LOG[before]
+        assert len(_parity.EXEMPT_LOG) == before + 1
+        assert rec["codes"] == x.numel() and n_diff == 0 and rec["differ"] == 0
+        assert rec["exempt_rel"] + rec["exempt_band_only"] == n_ex
+        assert n_ex <= _parity.rne_exempt_ceiling(128) * x.numel()
+        monkeypatch.setattr(_parity, "BOUNDARY_REL", 0.05)
+        with pytest.raises(AssertionError, match="ceiling"):
+            _parity.check_codes(gpu_codes, gpu_scales, codes, scales, t, qt, blk=128, axis=1)
+        del _parity.EXEMPT_LOG[before + 1:]  # the planted widening is not a parity record
+        monkeypatch.setattr(_parity, "BOUNDARY_REL", 1e-6)
