@@ -192,15 +192,21 @@ halo_status_t device_setup(int* dev_out) {
 
 // Device address of g_noalloc_scratch, one per device, set on the first
 // halo_linear_fwd_noalloc call made with that device current.
-void* g_noalloc_ptr[kMaxDevices] = {};
+// Read without the lock on the fast path, so atomic: a thread that sees a
+// non-null address (acquire) also sees the set-up that produced it (release).
+std::atomic<void*> g_noalloc_ptr[kMaxDevices] = {};
 
-halo_status_t noalloc_setup(int dev) {
-  if (g_noalloc_ptr[dev]) return HALO_OK;
-  std::lock_guard<std::mutex> lock(g_dev_mutex);
-  if (g_noalloc_ptr[dev]) return HALO_OK;
-  void* p = nullptr;
-  HALO_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-  g_noalloc_ptr[dev] = p;
+halo_status_t noalloc_setup(int dev, void** out) {
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      HALO_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
   return HALO_OK;
 }
 
@@ -1007,6 +1013,9 @@ halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, in
   if (!valid_qtype(qtype) || !valid_otype(otype)) return HALO_ERR_DTYPE;
   if (blk != 128 && blk != 256) return HALO_ERR_BLOCK;
   if (m <= 0 || n <= 0 || k <= 0 || pad_to(k, blk) > 32768) return HALO_ERR_SHAPE;
+  const int64_t esz = otype == HALO_OUT_FP32 ? 4 : 2;
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y) || (n * esz) % 16 != 0 || k % 8 != 0)
+    return HALO_ERR_ALIGN;
   const size_t need = ws_layout(m, n, k, 0, blk).total;
   if (need > HALO_NOALLOC_SCRATCH_BYTES) {
     snprintf(g_last_detail, sizeof g_last_detail,
@@ -1017,9 +1026,9 @@ halo_status_t halo_linear_fwd_noalloc(const void* x_bf16, const void* w_bf16, in
   int dev = 0;
   halo_status_t st = device_setup(&dev);
   if (st != HALO_OK) return st;
-  if ((st = noalloc_setup(dev)) != HALO_OK) return st;
-  return halo_linear_fwd(x_bf16, w_bf16, m, n, k, blk, qtype, y, otype, g_noalloc_ptr[dev],
-                         HALO_NOALLOC_SCRATCH_BYTES, stream);
+  void* scratch = nullptr;
+  if ((st = noalloc_setup(dev, &scratch)) != HALO_OK) return st;
+  return halo_linear_fwd(x_bf16, w_bf16, m, n, k, blk, qtype, y, otype, scratch, HALO_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 static halo_status_t linear_bwd_impl(const void* dy_bf16, const void* x_bf16, const void* w_bf16, int64_t m,

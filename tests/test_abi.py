@@ -134,6 +134,23 @@ def test_linear_host_validation(lib):
     assert b(FAKE, FAKE, FAKE, 256, 256, 512, 128, 0, FAKE, 0, FAKE, 0, FAKE, wsb - 1, None) == WORKSPACE
 
 
+def test_linear_fwd_noalloc_host_validation(lib):
+    """Every argument check of the scratch-free forward runs before it looks up
+    its device or the static array (here, with no GPU, that look-up would fail
+    with a CUDA status instead)."""
+    f = lib.halo_linear_fwd_noalloc
+    assert f(None, FAKE, 256, 256, 512, 128, 0, FAKE, 0, None) == NULL
+    assert f(FAKE, FAKE, 256, 256, 512, 64, 0, FAKE, 0, None) == BLOCK
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 9, FAKE, 0, None) == DTYPE
+    assert f(FAKE, FAKE, 256, 256, 32776, 128, 0, FAKE, 0, None) == SHAPE
+    assert f(MISALIGNED, FAKE, 256, 256, 512, 128, 0, FAKE, 0, None) == ALIGN
+    assert f(FAKE, MISALIGNED, 256, 256, 512, 128, 0, FAKE, 0, None) == ALIGN
+    assert f(FAKE, FAKE, 256, 256, 512, 128, 0, MISALIGNED, 0, None) == ALIGN
+    assert f(FAKE, FAKE, 256, 6, 512, 128, 0, FAKE, 1, None) == ALIGN     # 12-byte bf16 output rows
+    assert f(FAKE, FAKE, 256, 256, 500, 128, 0, FAKE, 0, None) == ALIGN   # 1000-byte rows of X
+    assert f(FAKE, FAKE, 8192, 8192, 4096, 128, 0, FAKE, 0, None) == WORKSPACE  # beyond the static scratch
+
+
 def test_hadamard_quantize_ex_host_validation(lib):
     f = lib.halo_hadamard_quantize_ex
     # plain arguments are checked as for halo_hadamard_quantize

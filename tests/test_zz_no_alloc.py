@@ -16,6 +16,7 @@ import torch
 
 import hadamard_rotated_precision_halo_b200 as halo
 from hadamard_rotated_precision_halo_b200 import inputs
+import oracle
 from tests._parity import check_output
 
 pytestmark = pytest.mark.gpu
@@ -41,14 +42,16 @@ def test_noalloc_forward_matches_workspace_forward(qtype, otype):
     w = inputs.weights(n, k, seed=62, device="cuda")
     ref = halo.halo_linear_fwd(x, w, blk, qtype, otype)  # the existing entry point, caller workspace
     torch.cuda.synchronize()
-    ref_np = ref.float().cpu().numpy().astype(np.float64)
     out_dtype = torch.float32 if otype == halo.HALO_OUT_FP32 else torch.bfloat16
     for _ in range(2):  # the second call finds the first call's codes still in the array
         y = torch.full((m, n), float("nan"), dtype=out_dtype, device="cuda")
         st = _call(lib, x, w, y, blk, qtype, otype)
         assert st == halo.HALO_OK, halo.status_text(st)
         torch.cuda.synchronize()
-        check_output(y, ref_np)
+        # the same kernels on the same inputs: bit for bit the workspace call's output
+        assert torch.equal(y, ref)
+    # and within the parity bar of the oracle
+    check_output(y, oracle.linear_fwd(x.cpu(), w.cpu(), blk, qtype))
     st, site = halo.halo_device_error()
     assert st == halo.HALO_OK, f"bounded wait ran out at site {site:#x}"
 
@@ -62,3 +65,16 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
                                      halo.HALO_Q_INT8, ctypes.c_void_p(x.data_ptr()), halo.HALO_OUT_FP32, None)
     assert st == halo.HALO_ERR_WORKSPACE
     assert b"scratch" in lib.halo_last_error_detail()
+
+
+def test_noalloc_rejects_misaligned_pointers_before_touching_the_device():
+    lib = halo.lib()
+    buf = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+    p = buf.data_ptr()
+    st = lib.halo_linear_fwd_noalloc(ctypes.c_void_p(p + 2), ctypes.c_void_p(p), 16, 16, 128, 128,
+                                     halo.HALO_Q_INT8, ctypes.c_void_p(p), halo.HALO_OUT_FP32, None)
+    assert st == halo.HALO_ERR_ALIGN
+    st = lib.halo_linear_fwd_noalloc(ctypes.c_void_p(p), ctypes.c_void_p(p), 16, 6, 128, 128, halo.HALO_Q_INT8,
+                                     ctypes.c_void_p(p), halo.HALO_OUT_BF16, None)  # a 12-byte output row
+    assert st == halo.HALO_ERR_ALIGN
+    assert torch.all(buf == 0)
