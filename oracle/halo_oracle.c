@@ -15,9 +15,8 @@
  *     (x[j], x[j+h]) <- (x[j]+x[j+h], x[j]-x[j+h]) for h = 1, 2, 4, ... and a
  *     final division by sqrt(n)  [QWHA page, sec. 2.1 "mathematical basis" and
  *     sec. 2.2 walsh_hadamard_transform].  Applied block-locally (blocks of b
- *     consecutive elements along the contraction dimension) as the HALO blog
- *     page's sec. 5 ("local rather than global Hadamard") and the QWHA page's
- *     sec. 5 (split very large dimensions into blocks) describe.
+ *     consecutive elements along the contraction dimension), the block-wise
+ *     reading of the HALO blog page, sec. 5, and of the QWHA page, sec. 5.
  *   - Symmetric absmax quantiser: scale = max|x| / qmax, qmax = 2^(bits-1)-1,
  *     q = clip(round(x / scale), -qmax, qmax), round = half-to-even
  *     [QWHA page, sec. 2.2 quantize]; FP8 E4M3 as the alternative 8-bit type
@@ -265,9 +264,8 @@ void halo_oracle_quantize(const double* v, int64_t rows, int64_t cols, int axis,
   }
 }
 
-/* Stochastic-rounding variant of the quantiser [QWHA page sec. 5: random
- * rounding reduces the bias of quantisation, floor(x) + (rand < x - floor(x))].
- * Same scale as above; the code of element idx rounds t = v / s to one of its
+/* Stochastic-rounding variant of the quantiser [QWHA page, sec. 5].  Same
+ * scale as above; the code of element idx rounds t = v / s to one of its
  * two grid neighbours lo <= t < hi, taking hi when u < (t - lo) / (hi - lo),
  * with u = rand[idx] / 65536 (16 caller-supplied random bits per element).
  * INT8 grid: the integers, clamped to +-127.  E4M3 grid: the E4M3 values,
