@@ -14,8 +14,11 @@ including the rotation and quantisation launches) over the device-timed
 steps, which replay the step's launches as one captured CUDA graph
 (`--no-graph`: launched from the host); rotate+quantise GB/s and the GEMM
 kernels' own TOPS are reported beside it, and `e2e` times the same step through
-the linear-layer calls with host buffers.  `--qtype e4m3` runs FP8, `--group
-64|128` group-wise scales.  `--impl reference` times the CPU oracle on a
+the linear-layer calls with host buffers.  The same line carries the other
+workloads measured on their own (`configs`): the tiny forward, rotate+quantise
+of [16384, 4096] activations, the Llama-7B attention-projection forward and
+FFN down-projection backward (INT8 and E4M3), and the 70B layer in E4M3.
+`--qtype e4m3` runs FP8 as the headline, `--group 64|128` group-wise scales.  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload instead.  `--measure-peaks` and
 `--rotq-shapes` print the GEMM peak comparison and the per-shape
 rotate+quantise table.
@@ -41,12 +44,25 @@ from hadamard_rotated_precision_halo_b200 import inputs  # noqa: E402
 
 METRIC = "rotated-qGEMM TOPS & rotate+quant GB/s at Llama shapes vs B200 peak (1 GPU)"
 # DRAM bytes (read + write) per qgemm_pair_kernel launch, averaged over the 21
-# GEMMs of the INT8 layer step, from one ncu capture of the current kernel
-# (profiles/qgemm_pair_kernel_llama70b_layer_traffic.md).  Set to None when the
-# kernel changes until it is captured again.
+# GEMMs of the INT8 layer step, from one ncu capture, and the SHA-256 prefix of
+# the GEMM kernel source (csrc/qgemm.cuh) that capture ran.  The bench reports
+# the figure only while the source still hashes the same, null otherwise.
 GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER = 484.5e6
+GEMM_TRAFFIC_SOURCE_SHA = "e1950ef468ee1082"
 UNIT = "TOPS"
 BLK = 128
+# The sustained 8-bit denominator applies when the timed region lasts long
+# enough for the board to settle at its power cap; shorter regions run at the
+# burst clock.
+SUSTAINED_REGION_S = 2.0
+
+
+def gemm_source_sha() -> str:
+    import hashlib
+
+    path = os.path.join(ROOT, "hadamard_rotated_precision_halo_b200", "csrc", "qgemm.cuh")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def peaks():
@@ -210,6 +226,20 @@ class LayerStep:
                     q = torch.empty(x.shape, dtype=self.code_dt, device=self.dev)
                     sc = torch.empty(self.n_scales(x, ax), dtype=torch.float32, device=self.dev)
                     self.shared[key] = (q, sc)
+        # dY feeds dX (rotated along its columns) and dW (along its rows): when
+        # the step has both, its two code sets come from one call
+        # (halo_hadamard_quantize_both: the second rotation reads dY from L2),
+        # the dim-0 set into a buffer of its own, kept until the dW GEMM.
+        both = {}
+        if self.group == 0 and "dx" in self.kinds and "dw" in self.kinds:
+            for g in self.shapes.gemms:
+                dy = self.t["dy"][g.name]
+                key = (dy.data_ptr(), h.HALO_AXIS_ROWS)
+                if key not in self.shared:
+                    q = torch.empty(self.halo.codes_shape(dy.shape[0], dy.shape[1], h.HALO_AXIS_ROWS, BLK),
+                                    dtype=self.code_dt, device=self.dev)
+                    self.shared[key] = (q, torch.empty(dy.shape[1], dtype=torch.float32, device=self.dev))
+                both[dy.data_ptr()] = key
         plan, done = [], set()
         for kind, name, a, a_axis, b, b_axis, m, n, k, c in gem:
             operands = []
@@ -223,7 +253,12 @@ class LayerStep:
                 else:
                     q = self._codes(self.qa if slot == 0 else self.qb, x.shape[0], x.shape[1])
                     sc = self.sa if slot == 0 else self.sb
-                    plan.append(("rotq", x, ax, q, sc))
+                    if ax == h.HALO_AXIS_COLS and x.data_ptr() in both and both[x.data_ptr()] not in done:
+                        qc, scc = self.shared[both[x.data_ptr()]]
+                        plan.append(("both", x, q, sc, qc, scc))
+                        done.add(both[x.data_ptr()])
+                    else:
+                        plan.append(("rotq", x, ax, q, sc))
                 operands.append((q, sc, ax))
             plan.append(("gemm", operands[0], operands[1], m, n, k, c))
         self._plan = plan
@@ -243,7 +278,13 @@ class LayerStep:
                 ev = torch.cuda.Event(enable_timing=True)
                 ev.record(stream)
                 events.append(ev)
-            if op[0] == "rotq":
+            if op[0] == "both":
+                _, x, q, sc, qc, scc = op
+                st = L.halo_hadamard_quantize_both(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), BLK, self.qtype,
+                                                   h._ptr(q), q.stride(0), h._ptr(sc), h._ptr(qc), qc.stride(0),
+                                                   h._ptr(scc), sp)
+                h._check(st, "halo_hadamard_quantize_both")
+            elif op[0] == "rotq":
                 _, x, ax, q, sc = op
                 if self.group:
                     st = L.halo_hadamard_quantize_grouped(h._ptr(x), x.shape[0], x.shape[1], x.stride(0), ax, BLK,
@@ -270,13 +311,14 @@ class LayerStep:
             ev = torch.cuda.Event(enable_timing=True)
             ev.record(stream)
             events.append(ev)
-        return len(plan)
+        return self.launches_per_step()
 
     def attribute(self, events, steps):
-        """Per-launch durations from an instrumented run of `steps` steps:
-        (gemm ms, [rotq ms, elements] per axis)."""
+        """Per-call durations from an instrumented run of `steps` steps:
+        (gemm ms, [rotate+quantise ms, elements] per axis; key 2: both axes
+        from one halo_hadamard_quantize_both call)."""
         plan = self.plan()
-        gemm_ms, by_axis = 0.0, {0: [0.0, 0], 1: [0.0, 0]}
+        gemm_ms, by_axis = 0.0, {0: [0.0, 0], 1: [0.0, 0], 2: [0.0, 0]}
         per = len(plan) + 1
         for s_i in range(steps):
             evs = events[s_i * per:(s_i + 1) * per]
@@ -285,9 +327,14 @@ class LayerStep:
                 if op[0] == "gemm":
                     gemm_ms += dt
                 else:
-                    by_axis[op[2]][0] += dt
-                    by_axis[op[2]][1] += op[1].numel()
+                    ax = 2 if op[0] == "both" else op[2]
+                    by_axis[ax][0] += dt
+                    by_axis[ax][1] += op[1].numel()
         return gemm_ms, by_axis
+
+    def launches_per_step(self) -> int:
+        """Kernel launches of one step (a "both" call launches two)."""
+        return sum(2 if op[0] == "both" else 1 for op in self.plan())
 
     def rotq_bytes(self) -> int:
         """Algorithmic bytes of the step's rotate+quantise launches: bf16 in
@@ -298,6 +345,9 @@ class LayerStep:
             if op[0] == "rotq":
                 x, ax = op[1], op[2]
                 total += 3 * x.numel() + 4 * self.n_scales(x, ax)
+            elif op[0] == "both":  # one read, two code sets, a scale per row and per column
+                x = op[1]
+                total += 4 * x.numel() + 4 * (x.shape[0] + x.shape[1])
         return total
 
     def gemm_bytes(self) -> int:
@@ -648,6 +698,113 @@ def measure_rotq_shapes(repeats: int = 10):
     return {"measure": "rotate+quantise per shape", "block": BLK, "results": out}
 
 
+# ------------------------------------------------------------ the other workloads
+def capture_step(step: "LayerStep"):
+    """The step's launches captured once as a CUDA graph (warmed up first)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step.run()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    return graph
+
+
+def _timed(fn, reps: int, flush=None) -> list:
+    """Device time (ms) of each of `reps` calls of fn, CUDA events on the
+    current stream; `flush` (a buffer larger than L2) is overwritten before
+    every call, outside the timed interval."""
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return ts
+
+
+def measure_other_configs(pk: dict, reps: int = 20) -> dict:
+    """The remaining workloads, each on its own, after the headline step:
+    the tiny forward X[64,256] W[128,256] (block 256, INT8, fp32 Y; latency);
+    rotate+quantise of [16384, 4096] activations (INT8, E4M3, both from one
+    read; GB/s against the HBM copy peak); the Llama-7B attention-projection
+    forward 8192x4096x4096 and FFN down-projection backward (dX + dW,
+    8192x11008x4096), INT8 and E4M3, TOPS including every rotate+quantise
+    launch against the burst 8-bit peak; and the Llama-70B layer step in E4M3.
+    Every call writes a 512 MB buffer first (outside the timing), so no input
+    is served from L2.  Median over `reps` calls (10 steps for the 70B layer,
+    whose inputs exceed L2 several times)."""
+    import hadamard_rotated_precision_halo_b200 as halo
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    hbm = pk["hbm_gbs"]
+    peak8 = 2.0 * pk["bf16"]
+    med = lambda ts: sorted(ts)[len(ts) // 2]
+    out = {"peak_8bit_tops": peak8, "peak_hbm_gbs": hbm, "timing": f"median of {reps}, L2 flushed before each"}
+
+    # tiny forward (latency-bound: report the call's device time)
+    x = inputs.plain(64, 256, seed=0, device="cuda")
+    w = inputs.plain(128, 256, seed=1, device="cuda")
+    y = torch.empty((64, 128), dtype=torch.float32, device="cuda")
+    ws = torch.empty(halo.halo_workspace_size(64, 128, 256, 0), dtype=torch.uint8, device="cuda")
+    fn = lambda: halo.halo_linear_fwd(x, w, 256, halo.HALO_Q_INT8, halo.HALO_OUT_FP32, y=y, ws=ws)
+    for _ in range(3):
+        fn()
+    ms = med(_timed(fn, reps, flush))
+    out["tiny_fwd_64x128x256"] = {"us": ms * 1e3, "tops": 2 * 64 * 128 * 256 / (ms * 1e-3) / 1e12,
+                                  "launches": 3, "bound": "launch latency"}
+    del x, w, y, ws
+
+    # standalone rotate+quantise [16384, 4096]
+    x = inputs.activations(16384, 4096, seed=2, device="cuda")
+    rq = {}
+    for name, qt in (("int8", halo.HALO_Q_INT8), ("e4m3", halo.HALO_Q_E4M3)):
+        q, sc = halo.halo_hadamard_quantize(x, halo.HALO_AXIS_COLS, BLK, qt)
+        ms = med(_timed(lambda: halo.halo_hadamard_quantize(x, halo.HALO_AXIS_COLS, BLK, qt, q_out=q,
+                                                            scales_out=sc), reps, flush))
+        gb = (3 * x.numel() + 4 * sc.numel()) / (ms * 1e-3) / 1e9
+        rq[name] = {"us": ms * 1e3, "gbs": gb, "frac": gb / hbm}
+        del q, sc
+    outs = halo.halo_hadamard_quantize_dual(x, BLK)
+    ms = med(_timed(lambda: halo.halo_hadamard_quantize_dual(x, BLK, *outs), reps, flush))
+    gb = (4 * x.numel() + 8 * x.shape[0]) / (ms * 1e-3) / 1e9
+    rq["int8+e4m3_one_read"] = {"us": ms * 1e3, "gbs": gb, "frac": gb / hbm}
+    out["rotate_quantize_16384x4096"] = rq
+    del x, outs
+
+    # single-GEMM Llama-7B cases and the 70B layer in E4M3
+    cases = [("llama7b_attn_proj_fwd", "int8"), ("llama7b_attn_proj_fwd", "e4m3"),
+             ("llama7b_ffn_down_bwd", "int8"), ("llama7b_ffn_down_bwd", "e4m3"),
+             ("llama70b_layer_fwd_bwd", "e4m3")]
+    for wl, qname in cases:
+        shapes, kinds = WORKLOADS[wl]
+        qt = halo.HALO_Q_INT8 if qname == "int8" else halo.HALO_Q_E4M3
+        st = LayerStep(shapes, seed=4, device=torch.device("cuda"), qtype=qt, kinds=kinds)
+        g = capture_step(st)
+        if wl == "llama70b_layer_fwd_bwd":
+            ts = _timed(g.replay, 10)
+        else:
+            ts = _timed(g.replay, reps, flush)
+        ms = med(ts)
+        tops = st.ops_per_step() / (ms * 1e-3) / 1e12
+        out.setdefault(wl, {})[qname] = {"ms_per_step": ms, "tops": tops, "frac_burst": tops / peak8,
+                                         "target_frac": 0.60, "launches": st.launches_per_step()}
+        del g, st
+        torch.cuda.synchronize()
+    return out
+
+
 # ------------------------------------------------------------------ multi-rank
 def max_over_ranks(ms: float, world: int, device) -> float:
     """Device-timed region of this rank -> the maximum over all ranks (the
@@ -671,6 +828,7 @@ WORKLOADS = {
     "llama7b_attn_proj_fwd": (inputs.LLAMA7B_ATTN_PROJ, ("fwd",)),
     "llama7b_ffn_down_bwd": (inputs.LLAMA7B_FFN_DOWN, ("dx", "dw")),
     "llama70b_gate_proj_dx": (inputs.LLAMA70B_GATE, ("dx",)),
+    "llama70b_q_proj_dw": (inputs.LLAMA70B_Q, ("dw",)),
 }
 
 
@@ -687,6 +845,8 @@ def main():
                     help="launch every kernel from the host instead of replaying the captured step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the tiny, rotate+quantise, Llama-7B and FP8 70B-layer measurements")
     ap.add_argument("--workload", default="llama70b_layer_fwd_bwd", choices=sorted(WORKLOADS),
                     help="the bench line uses the default; the single-GEMM cases serve profiling")
     ap.add_argument("--measure-peaks", action="store_true",
@@ -779,7 +939,7 @@ def main():
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    per_step = len(step.plan())
+    per_step = step.launches_per_step()
     with ClockSampler(local) as clocks:
         start.record(stream)
         launches = 0
@@ -806,7 +966,7 @@ def main():
     torch.cuda.synchronize()
     gemm_ms, by_axis = step.attribute(events, args.steps)
     ms_instrumented = events[0].elapsed_time(events[-1]) / args.steps
-    rotq_ms = by_axis[0][0] + by_axis[1][0]
+    rotq_ms = by_axis[0][0] + by_axis[1][0] + by_axis[2][0]
     n_gemm = sum(1 for op in step.plan() if op[0] == "gemm") * args.steps
 
     ops_step = step.ops_per_step()
@@ -816,12 +976,17 @@ def main():
     rotq_gbs = step.rotq_bytes() * args.steps / (rotq_ms * 1e-3) / 1e9
     pk = peaks()
     # INT8 / FP8 dense peak: the measured bf16 cuBLAS figure times the nominal
-    # 8-bit : bf16 ratio (4.5 : 2.25); sustained figure, the GEMMs run inside a long step.
-    peak8 = 2.0 * pk["bf16_sustained"]
+    # 8-bit : bf16 ratio (4.5 : 2.25), burst or sustained by the timed region's length.
+    peak8_burst, peak8_sus = 2.0 * pk["bf16"], 2.0 * pk["bf16_sustained"]
+    region_s = ms_total * 1e-3
+    sustained = region_s >= SUSTAINED_REGION_S
+    peak8 = peak8_sus if sustained else peak8_burst
 
-    def gbs(axis):
-        return 3 * by_axis[axis][1] / max(by_axis[axis][0] * 1e-3, 1e-12) / 1e9
+    def gbs(axis):  # 3 B per element (bf16 in, code out); both axes from one read: 4 B
+        return (4 if axis == 2 else 3) * by_axis[axis][1] / max(by_axis[axis][0] * 1e-3, 1e-12) / 1e9
 
+    traffic_ok = (args.workload == "llama70b_layer_fwd_bwd" and args.qtype == "int8" and not args.group
+                  and GEMM_TRAFFIC_SOURCE_SHA is not None and gemm_source_sha() == GEMM_TRAFFIC_SOURCE_SHA)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8" if qtype == halo.HALO_Q_INT8 else "e4m3",
@@ -829,19 +994,30 @@ def main():
             "gpu_launches": launches,
             "roofline": {"bound": "tensor", "kernel": "qgemm_grouped_kernel" if args.group else "qgemm_pair_kernel",
                          "achieved": gemm_tops, "peak": peak8, "unit": "TFLOP/s", "frac": gemm_tops / peak8,
-                         "traffic": (GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER
-                                     if args.workload == "llama70b_layer_fwd_bwd" and args.qtype == "int8"
-                                     and not args.group else None),
+                         "peak_kind": "sustained" if sustained else "burst",
+                         "frac_burst": gemm_tops / peak8_burst, "frac_sustained": gemm_tops / peak8_sus,
+                         "peak_burst": peak8_burst, "peak_sustained": peak8_sus,
+                         "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER if traffic_ok else None,
                          "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                          "algorithmic_bytes_per_launch": step.gemm_bytes() / max(n_gemm // args.steps, 1),
-                         "peak_note": f"2 x {pk['source']} bf16 sustained ({pk['bf16_sustained']}); "
-                                      f"burst 2 x {pk['bf16']} = {2 * pk['bf16']:.1f}",
+                         "peak_note": f"2 x {pk['source']} bf16 dense (8-bit : bf16 = 2 : 1); "
+                                      f"{'sustained' if sustained else 'burst'} for a {region_s:.2f} s timed region",
                          "launches": n_gemm, "avg_launch_ms": gemm_ms / max(n_gemm, 1)},
+            "step_roofline": {"achieved": value / max(world, 1), "unit": "TFLOP/s", "peak": peak8,
+                              "frac": value / max(world, 1) / peak8,
+                              "frac_burst": value / max(world, 1) / peak8_burst,
+                              "frac_sustained": value / max(world, 1) / peak8_sus, "target_frac": 0.60,
+                              "note": "whole step per GPU, every rotate+quantise launch included"},
             "rotq": {"gbs": rotq_gbs, "peak_gbs": pk["hbm_gbs"], "frac": rotq_gbs / pk["hbm_gbs"],
+                     "target_frac": 0.70,
                      "bytes_per_step": step.rotq_bytes(), "ms_per_step": rotq_ms / args.steps,
                      "along_contiguous_dim_gbs": gbs(0), "along_dim0_gbs": gbs(1),
+                     "along_contiguous_dim_frac": gbs(0) / pk["hbm_gbs"], "along_dim0_frac": gbs(1) / pk["hbm_gbs"],
                      "along_contiguous_dim_ms_per_step": by_axis[0][0] / args.steps,
-                     "along_dim0_ms_per_step": by_axis[1][0] / args.steps},
+                     "along_dim0_ms_per_step": by_axis[1][0] / args.steps,
+                     "both_axes_of_dy_gbs": gbs(2) if by_axis[2][1] else None,
+                     "both_axes_of_dy_frac": gbs(2) / pk["hbm_gbs"] if by_axis[2][1] else None,
+                     "both_axes_of_dy_ms_per_step": by_axis[2][0] / args.steps},
             "ms_per_step_instrumented": ms_instrumented,
             "clocks": clocks.summary()}
 
@@ -854,6 +1030,9 @@ def main():
             line["e2e"] = {"value": job_throughput(ops_step, 1, world, e2e_ms), "unit": UNIT,
                            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                            "steps": e2e_steps, "copies": "own stream per direction, overlapped with the kernels"}
+    if (world == 1 and not args.no_other_configs and args.workload == "llama70b_layer_fwd_bwd"
+            and not args.group and args.qtype == "int8"):
+        line["configs"] = measure_other_configs(pk)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if world > 1:

@@ -51,6 +51,9 @@ EXPORTS = (
     "halo_linear_fwd",
     "halo_linear_bwd",
     "halo_linear_fwd_noalloc",
+    "halo_hadamard_colmax",
+    "halo_hadamard_quantize_both",
+    "halo_hadamard_quantize_colmax",
     "halo_status_string",
     "halo_device_error",
     "halo_selftest_wait_timeout",
@@ -110,6 +113,12 @@ def lib():
     L.halo_linear_bwd.restype = I
     L.halo_linear_fwd_noalloc.argtypes = [P, P, I64, I64, I64, I, I, P, I, P]
     L.halo_linear_fwd_noalloc.restype = I
+    L.halo_hadamard_quantize_both.argtypes = [P, I64, I64, I64, I, I, P, I64, P, P, I64, P, P]
+    L.halo_hadamard_quantize_both.restype = I
+    L.halo_hadamard_colmax.argtypes = [P, I64, I64, I64, I, P, P]
+    L.halo_hadamard_colmax.restype = I
+    L.halo_hadamard_quantize_colmax.argtypes = [P, I64, I64, I64, I, I, P, P, I64, P, P]
+    L.halo_hadamard_quantize_colmax.restype = I
     L.halo_status_string.argtypes = [I]
     L.halo_status_string.restype = ctypes.c_char_p
     L.halo_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -196,6 +205,50 @@ def halo_hadamard_quantize_ex(x: torch.Tensor, axis: int, blk: int, qtype: int, 
                                          _ptr(rand_bits), ld_rand, _ptr(q_out), q_out.stride(0), _ptr(scales_out),
                                          _stream(stream))
     _check(st, "halo_hadamard_quantize_ex")
+    return q_out, scales_out
+
+
+def halo_hadamard_quantize_both(x: torch.Tensor, blk: int, qtype: int, outs=None, stream=None):
+    """Both code sets of x, rotated along the contiguous dimension (per-row
+    scales) and along dimension 0 (per-column scales), the second rotation
+    reading x from L2; returns (q_rows, scales_rows, q_cols, scales_cols)."""
+    rows, cols = x.shape
+    if outs is None:
+        outs = (torch.empty(codes_shape(rows, cols, HALO_AXIS_COLS, blk), dtype=_code_dtype(qtype), device=x.device),
+                torch.empty(rows, dtype=torch.float32, device=x.device),
+                torch.empty(codes_shape(rows, cols, HALO_AXIS_ROWS, 128), dtype=_code_dtype(qtype), device=x.device),
+                torch.empty(cols, dtype=torch.float32, device=x.device))
+    qr, sr, qc, sc = outs
+    _check(lib().halo_hadamard_quantize_both(_ptr(x), rows, cols, x.stride(0), blk, qtype, _ptr(qr), qr.stride(0),
+                                             _ptr(sr), _ptr(qc), qc.stride(0), _ptr(sc), _stream(stream)),
+           "halo_hadamard_quantize_both")
+    return outs
+
+
+def halo_hadamard_colmax(x: torch.Tensor, blk: int = 128, amax_out=None, stream=None) -> torch.Tensor:
+    """Per-column maxima of |H_128 x| (unnormalised block transform along
+    dimension 0) over the rows of x: fp32 [cols]."""
+    rows, cols = x.shape
+    if amax_out is None:
+        amax_out = torch.empty(cols, dtype=torch.float32, device=x.device)
+    _check(lib().halo_hadamard_colmax(_ptr(x), rows, cols, x.stride(0), blk, _ptr(amax_out), _stream(stream)),
+           "halo_hadamard_colmax")
+    return amax_out
+
+
+def halo_hadamard_quantize_colmax(x: torch.Tensor, blk: int, qtype: int, amax: torch.Tensor, q_out=None,
+                                  scales_out=None, stream=None):
+    """Codes and scales of x rotated along dimension 0 with given per-column
+    maxima (halo_hadamard_colmax merged over every holder of x's rows)."""
+    rows, cols = x.shape
+    shape = codes_shape(rows, cols, HALO_AXIS_ROWS, blk)
+    if q_out is None:
+        q_out = torch.empty(shape, dtype=_code_dtype(qtype), device=x.device)
+    if scales_out is None:
+        scales_out = torch.empty(cols, dtype=torch.float32, device=x.device)
+    _check(lib().halo_hadamard_quantize_colmax(_ptr(x), rows, cols, x.stride(0), blk, qtype, _ptr(amax), _ptr(q_out),
+                                               q_out.stride(0), _ptr(scales_out), _stream(stream)),
+           "halo_hadamard_quantize_colmax")
     return q_out, scales_out
 
 

@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -117,6 +118,37 @@ Cols1Kernel cols_1pass_kernel(int qtype, int nw, bool ext) {
   return ext ? cols_1pass_for<1, 1>(nw) : cols_1pass_for<1, 0>(nw);
 }
 
+// Dimension-0 rotation with the rotated values parked in tensor memory:
+// variant 0 (<= 64 blocks of 128 rows): 4 warps, two strips in tensor memory;
+// variant 1 (<= 128 blocks): 8 warps, two strips; variant 2 (<= 256 blocks):
+// 8 warps of two blocks each, one strip.
+typedef void (*ColsTmKernel)(const CUtensorMap, const CUtensorMap, RotqColsTmParams);
+constexpr int kColsTmVariants = 3;
+constexpr int kColsTmWarps[kColsTmVariants] = {4, 8, 8};
+constexpr int kColsTmBlocksPerCta[kColsTmVariants] = {4, 8, 16};
+
+template <int QT, int EXT>
+ColsTmKernel cols_tm_for(int variant) {
+  switch (variant) {
+    case 0: return rotq_cols_tm_kernel<QT, 4, 2, 1, EXT>;
+    case 1: return rotq_cols_tm_kernel<QT, 8, 2, 1, EXT>;
+    default: return rotq_cols_tm_kernel<QT, 8, 1, 2, EXT>;
+  }
+}
+
+// ext: random signs and / or stochastic rounding (RotqExtras).
+ColsTmKernel cols_tm_kernel(int qtype, int variant, bool ext) {
+  if (qtype == HALO_Q_INT8) return ext ? cols_tm_for<0, 1>(variant) : cols_tm_for<0, 0>(variant);
+  return ext ? cols_tm_for<1, 1>(variant) : cols_tm_for<1, 0>(variant);
+}
+
+typedef void (*ColsSplitKernel)(const CUtensorMap, const CUtensorMap, RotqColsSplitParams);
+
+ColsSplitKernel cols_split_kernel(int qtype, int mode) {
+  if (mode == 0) return rotq_cols_split_kernel<0, 0>;  // maxima only: no codes, the type does not matter
+  return qtype == HALO_Q_INT8 ? rotq_cols_split_kernel<0, 1> : rotq_cols_split_kernel<1, 1>;
+}
+
 Cols2Kernel cols_2pass_kernel(int qtype, bool ext) {
   if (qtype == HALO_Q_INT8) return ext ? rotq_cols_kernel<0, 1> : rotq_cols_kernel<0, 0>;
   return ext ? rotq_cols_kernel<1, 1> : rotq_cols_kernel<1, 0>;
@@ -171,6 +203,17 @@ halo_status_t device_setup(int* dev_out) {
         }
       }
     }
+    HALO_CUDA(set_smem_attr(cols_split_kernel(0, 0), optin));
+    HALO_CUDA(set_smem_attr(cols_split_kernel(0, 1), optin));
+    HALO_CUDA(set_smem_attr(cols_split_kernel(1, 1), optin));
+    for (int qt = 0; qt < 2; ++qt) {
+      for (int v = 0; v < kColsTmVariants; ++v) {
+        for (int e = 0; e < 2; ++e) {
+          HALO_CUDA(set_smem_attr(cols_tm_kernel(qt, v, e), optin));
+          HALO_CUDA(cudaFuncSetAttribute(cols_tm_kernel(qt, v, e), cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        }
+      }
+    }
     for (int e = 0; e < 2; ++e) {
       for (int qt = 0; qt < 2; ++qt) {
         HALO_CUDA(set_smem_attr(cols_2pass_kernel(qt, e), optin));
@@ -185,6 +228,10 @@ halo_status_t device_setup(int* dev_out) {
     HALO_CUDA(set_smem_attr(qgemm_kernel<1>, optin));
     HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 1, 0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 1, 1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 1, 0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 1, 1>, optin));
   }
   d.ready.store(true, std::memory_order_release);
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
@@ -239,6 +286,22 @@ struct Launch {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// EXPERIMENT ONLY (removed before commit): A/B switch for the tensor-memory dim-0 kernel.
+static const bool g_cols_tm_enabled = [] {
+  const char* e = getenv("HALO_COLS_TM");
+  return !(e && e[0] == '0');
+}();
+// EXPERIMENT ONLY (removed before commit): raster group of the pair GEMM.
+static const int g_gemm_group_m = [] {
+  const char* e = getenv("HALO_GEMM_GROUPM");
+  return e && atoi(e) > 0 ? atoi(e) : 16;
+}();
+// EXPERIMENT ONLY (removed before commit): A/B switch for the bulk-store GEMM epilogue.
+static const bool g_gemm_staged = [] {
+  const char* e = getenv("HALO_GEMM_STAGED");
+  return !(e && e[0] == '0');
+}();
 
 halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
                      const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle sw) {
@@ -465,12 +528,64 @@ halo_status_t launch_rotq_cols_1pass(const void* x, int64_t rows, int64_t cols, 
   return HALO_OK;
 }
 
+// Rotation along dimension 0 of up to 256 blocks of 128 rows, the rotated
+// values parked in tensor memory across the cluster's column-max reduction
+// (rotq_cols_tm_kernel).  One CTA per SM for the 8-warp variants (all of the
+// SM's tensor memory), two for the 4-warp one.
+halo_status_t launch_rotq_cols_tm(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
+                                  int64_t ld_q, float* scales, const RotqExtras& ex, bool ext, cudaStream_t stream,
+                                  int variant, int nblocks, int dev) {
+  const int strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
+  const int cl = (nblocks + kColsTmBlocksPerCta[variant] - 1) / kColsTmBlocksPerCta[variant];
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(pad_to(rows, 128))};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  RotqColsTmParams p;
+  p.scales = scales;
+  p.cols = cols;
+  p.strips = strips;
+  p.nblocks = nblocks;
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  p.ex = ex;
+  ColsTmKernel kern = cols_tm_kernel(qtype, variant, ext);
+  // Persistent: as many clusters as fit at once (each loops over strips).
+  Launch L(dim3(cl, 1, 1), dim3(32 * kColsTmWarps[variant]), cols_tm_smem(kColsTmWarps[variant]), stream, cl);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &L.cfg) != cudaSuccess || max_clusters < 1) {
+    (void)cudaGetLastError();
+    max_clusters = std::max(1, g_dev[dev].sm_count / cl);
+  }
+  L.cfg.gridDim = dim3(cl, std::min(strips, max_clusters), 1);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
 halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, void* q,
                                int64_t ld_q, float* scales, const RotqExtras& ex, bool ext, cudaStream_t stream,
                                int dev) {
   // Rows past the input (zero padding to whole 128-row blocks) are outside the
   // input tensor map and arrive as zeros; the codes cover the padded rows.
   const int nblocks = static_cast<int>(pad_to(rows, 128) / 128);
+  if (g_cols_tm_enabled) {
+    for (int v = 0; v < kColsTmVariants; ++v)
+      if (nblocks <= 16 * kColsTmBlocksPerCta[v])
+        return launch_rotq_cols_tm(x, rows, cols, ld_x, qtype, q, ld_q, scales, ex, ext, stream, v, nblocks, dev);
+  }
   // Most warps per CTA (up to 4) with at most 16 CTAs per cluster.
   for (int nw = 4; nw >= 1; --nw) {
     if (nblocks % nw == 0 && nblocks / nw <= 16)
@@ -545,6 +660,53 @@ halo_status_t launch_rotq_cols_grouped(const void* x, int64_t rows, int64_t cols
   p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
   p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
   ColsGrKernel kern = qtype == HALO_Q_INT8 ? rotq_cols_grouped_kernel<0> : rotq_cols_grouped_kernel<1>;
+  const size_t smem = 4 * (2 * kColsInBytes) + 128;
+  int per_sm = 0;
+  HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, smem));
+  if (per_sm < 1) per_sm = 1;
+  const int64_t items = static_cast<int64_t>(p.nblocks) * p.strips;
+  const int grid = static_cast<int>(std::min<int64_t>((items + 3) / 4, static_cast<int64_t>(g_dev[dev].sm_count) * per_sm));
+  Launch L(dim3(grid), dim3(128), smem, stream, 0);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_x, tm_q, p));
+  return HALO_OK;
+}
+
+// Dimension-0 rotation split at the column maxima (rotq_cols_split_kernel):
+// mode 0 merges this matrix's per-column maxima into amax (zeroed here first),
+// mode 1 writes codes and scales from given maxima.  Independent warps over
+// the (128-row block, 32-column strip) items.
+halo_status_t launch_rotq_cols_split(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int qtype, int mode,
+                                     float* amax, void* q, int64_t ld_q, float* scales, cudaStream_t stream,
+                                     int dev) {
+  CUtensorMap tm_x, tm_q;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  }
+  if (mode == 1) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(pad_to(rows, 128))};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_q)};
+    cuuint32_t box[2] = {kColsStrip, 128};
+    halo_status_t st = encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != HALO_OK) return st;
+  } else {
+    tm_q = tm_x;  // never used: mode 0 stores no codes
+    HALO_CUDA(cudaMemsetAsync(amax, 0, static_cast<size_t>(cols) * sizeof(float), stream));
+  }
+  RotqColsSplitParams p;
+  p.amax = amax;
+  p.scales = scales;
+  p.cols = cols;
+  p.strips = static_cast<int>((cols + kColsStrip - 1) / kColsStrip);
+  p.nblocks = static_cast<int>(pad_to(rows, 128) / 128);
+  p.qmax = qtype == HALO_Q_INT8 ? 127.f : 448.f;
+  p.scale_mult = static_cast<float>(1.0 / (static_cast<double>(p.qmax) * sqrt(128.0)));
+  ColsSplitKernel kern = cols_split_kernel(qtype, mode);
   const size_t smem = 4 * (2 * kColsInBytes) + 128;
   int per_sm = 0;
   HALO_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, smem));
@@ -668,6 +830,7 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.a_mn = a_mn;
   p.b_mn = b_mn;
+  p.group_m = g_gemm_group_m;
   // Instruction descriptor: D format (bits 4-5), A/B formats (7-9, 10-12),
   // A/B major (15, 16), N >> 3 (17-22), M >> 4 (24-28).
   uint32_t idesc = 0;
@@ -695,11 +858,27 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
     return HALO_OK;
   }
   const int pairs = std::min(p.num_tiles, g_dev[dev].sm_count / 2);
-  Launch L(dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, stream, 2);
-  if (qtype == HALO_Q_INT8)
-    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_pair_kernel<0>, tm_a, tm_b, p));
+  // The output as a tensor for the bulk-store epilogue: 32 rows x 128 bytes
+  // per copy, 128-byte swizzle (the layout the epilogue writes).
+  const bool bf16_out = otype == HALO_OUT_BF16;
+  CUtensorMap tm_c;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(m)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_c) * (bf16_out ? 2 : 4)};
+    cuuint32_t box[2] = {bf16_out ? 64u : 32u, 32u};
+    halo_status_t st = encode(&tm_c, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                              c, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != HALO_OK) return st;
+  }
+  typedef void (*PairKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, GemmParams);
+  PairKernel kern;
+  if (g_gemm_staged)
+    kern = qtype == HALO_Q_INT8 ? (bf16_out ? qgemm_pair_kernel<0, 1, 1> : qgemm_pair_kernel<0, 1, 0>)
+                                : (bf16_out ? qgemm_pair_kernel<1, 1, 1> : qgemm_pair_kernel<1, 1, 0>);
   else
-    HALO_CUDA(cudaLaunchKernelEx(&L.cfg, qgemm_pair_kernel<1>, tm_a, tm_b, p));
+    kern = qtype == HALO_Q_INT8 ? qgemm_pair_kernel<0> : qgemm_pair_kernel<1>;
+  Launch L(dim3(2 * pairs), dim3(kGemmThreads), g_gemm_staged ? kPairSmemBytesStaged : kPairSmemBytes, stream, 2);
+  HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_a, tm_b, tm_c, p));
   return HALO_OK;
 }
 
@@ -879,6 +1058,25 @@ halo_status_t halo_hadamard_quantize(const void* x_bf16, int64_t rows, int64_t c
                                    scales_out, stream);
 }
 
+halo_status_t halo_hadamard_quantize_both(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
+                                          int qtype, void* q_rows, int64_t ld_qr, float* scales_rows, void* q_cols,
+                                          int64_t ld_qc, float* scales_cols, void* stream) {
+  // Every argument of both rotations is checked before either is launched.
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_COLS, blk, qtype, q_rows, ld_qr,
+                                             scales_rows);
+  if (st != HALO_OK) return st;
+  if ((st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_ROWS, 128, qtype, q_cols, ld_qc,
+                                    scales_cols)) != HALO_OK)
+    return st;
+  // Back to back on the stream: the second rotation reads X while the first
+  // has just brought it through L2.
+  if ((st = halo_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_COLS, blk, qtype, q_rows, ld_qr, scales_rows,
+                                   stream)) != HALO_OK)
+    return st;
+  return halo_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_ROWS, 128, qtype, q_cols, ld_qc, scales_cols,
+                                stream);
+}
+
 halo_status_t halo_hadamard_quantize_dual(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
                                           void* q_int8, int64_t ld_q8, float* scales_int8, void* q_e4m3,
                                           int64_t ld_qf8, float* scales_e4m3, void* stream) {
@@ -918,6 +1116,33 @@ halo_status_t halo_hadamard_quantize_grouped(const void* x_bf16, int64_t rows, i
                             nullptr, 0, nullptr, group);
   }
   return launch_rotq_cols_grouped(x_bf16, rows, cols, ld_x, qtype, q_out, ld_q, scales_out, group, s, dev);
+}
+
+halo_status_t halo_hadamard_colmax(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
+                                   float* amax_out, void* stream) {
+  // The checks of halo_hadamard_quantize along dimension 0 (amax_out stands in
+  // for the codes and scales, which this call does not write).
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_ROWS, blk, HALO_Q_INT8, amax_out,
+                                             cols + (16 - cols % 16) % 16, amax_out);
+  if (st != HALO_OK) return st;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != HALO_OK) return st;
+  return launch_rotq_cols_split(x_bf16, rows, cols, ld_x, HALO_Q_INT8, 0, amax_out, nullptr, 0, nullptr,
+                                static_cast<cudaStream_t>(stream), dev);
+}
+
+halo_status_t halo_hadamard_quantize_colmax(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
+                                            int qtype, const float* amax, void* q_out, int64_t ld_q,
+                                            float* scales_out, void* stream) {
+  halo_status_t st = check_hadamard_quantize(x_bf16, rows, cols, ld_x, HALO_AXIS_ROWS, blk, qtype, q_out, ld_q,
+                                             scales_out);
+  if (st != HALO_OK) return st;
+  if (!amax) return HALO_ERR_NULL;
+  if (!aligned16(amax)) return HALO_ERR_ALIGN;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != HALO_OK) return st;
+  return launch_rotq_cols_split(x_bf16, rows, cols, ld_x, qtype, 1, const_cast<float*>(amax), q_out, ld_q,
+                                scales_out, static_cast<cudaStream_t>(stream), dev);
 }
 
 halo_status_t halo_qgemm_grouped(const void* a_q, const float* s_a, int a_major, int64_t ld_a, const void* b_q,
@@ -1054,6 +1279,13 @@ static halo_status_t linear_bwd_impl(const void* dy_bf16, const void* x_bf16, co
   if (dw && (k * (otype_dw == HALO_OUT_FP32 ? 4 : 2)) % 16 != 0) return HALO_ERR_ALIGN;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   halo_status_t st;
+  // With both products, dY is rotated both ways back to back (the second
+  // rotation reads it from L2 when it fits there), before W and X.
+  const bool both = dx && dw && group == 0;
+  if (both && (st = halo_hadamard_quantize_both(dy_bf16, m, n, n, blk, qtype, w8 + L.off[0], pad_to(n, blk),
+                                                reinterpret_cast<float*>(w8 + L.off[2]), w8 + L.off[4], n,
+                                                reinterpret_cast<float*>(w8 + L.off[6]), stream)) != HALO_OK)
+    return st;
   if (dx) {
     uint8_t* dyq = w8 + L.off[0];
     uint8_t* wq = w8 + L.off[1];
@@ -1061,7 +1293,8 @@ static halo_status_t linear_bwd_impl(const void* dy_bf16, const void* x_bf16, co
     float* sw = reinterpret_cast<float*>(w8 + L.off[3]);
     // dX[M,K] = dY[M,N] W[N,K]: contraction over N (zero-padded to np).
     const int64_t np = pad_to(n, blk);
-    if ((st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, group, qtype, dyq, np, sdy, stream)) != HALO_OK)
+    if (!both &&
+        (st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_COLS, blk, group, qtype, dyq, np, sdy, stream)) != HALO_OK)
       return st;
     if ((st = quantize_op(w_bf16, n, k, k, HALO_AXIS_ROWS, blk, group, qtype, wq, k, sw, stream)) != HALO_OK)
       return st;
@@ -1076,7 +1309,8 @@ static halo_status_t linear_bwd_impl(const void* dy_bf16, const void* x_bf16, co
     float* sx = reinterpret_cast<float*>(w8 + L.off[7]);
     // dW[N,K] = dY^T[N,M] X[M,K]: contraction over M (tokens, zero-padded to mp).
     const int64_t mp = pad_to(m, blk);
-    if ((st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, group, qtype, dyq, n, sdy, stream)) != HALO_OK)
+    if (!both &&
+        (st = quantize_op(dy_bf16, m, n, n, HALO_AXIS_ROWS, blk, group, qtype, dyq, n, sdy, stream)) != HALO_OK)
       return st;
     if ((st = quantize_op(x_bf16, m, k, k, HALO_AXIS_ROWS, blk, group, qtype, xq, k, sx, stream)) != HALO_OK)
       return st;

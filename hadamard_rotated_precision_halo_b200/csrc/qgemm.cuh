@@ -50,6 +50,7 @@ struct GemmParams {
   int m, n, k;
   int tiles_m, tiles_n, num_tiles;
   int a_mn, b_mn;  // operand storage: 0 = K-major, 1 = MN-major
+  int group_m;     // tile raster of the pair kernel (M tiles per group)
   uint32_t idesc;  // tcgen05 instruction descriptor
   const float* sa;
   const float* sb;
@@ -58,14 +59,21 @@ struct GemmParams {
   int out_bf16;
 };
 
-__device__ __forceinline__ void gemm_tile_coords(int tile, int tiles_m, int tiles_n, int& tm, int& tn) {
-  const int per_group = kGemmGroupM * tiles_n;
+// Tile raster: groups of `group_m` M tiles; inside a group the M tiles of one
+// N column come one after another, so that consecutive tiles (computed at the
+// same time by neighbouring CTAs) share B panels and the group's A panels.
+__device__ __forceinline__ void gemm_tile_coords(int tile, int tiles_m, int tiles_n, int group_m, int& tm, int& tn) {
+  const int per_group = group_m * tiles_n;
   const int group = tile / per_group;
-  const int first_m = group * kGemmGroupM;
-  const int gm = min(tiles_m - first_m, kGemmGroupM);
+  const int first_m = group * group_m;
+  const int gm = min(tiles_m - first_m, group_m);
   const int in_group = tile - group * per_group;
   tm = first_m + in_group % gm;
   tn = in_group / gm;
+}
+
+__device__ __forceinline__ void gemm_tile_coords(int tile, int tiles_m, int tiles_n, int& tm, int& tn) {
+  gemm_tile_coords(tile, tiles_m, tiles_n, kGemmGroupM, tm, tn);
 }
 
 template <int QT>
@@ -277,6 +285,10 @@ constexpr int kPairStages = 6;
 constexpr int kPairABytes = 128 * kGemmBK;  // 16 KB: 128 rows of A
 constexpr int kPairBBytes = 128 * kGemmBK;  // 16 KB: 128 N indices of B
 constexpr size_t kPairSmemBytes = kPairStages * (kPairABytes + kPairBBytes) + 1024 + 256;
+// Output staging of the bulk-store epilogue: per epilogue warp two buffers of
+// 32 rows x 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzled.
+constexpr int kPairOutBytes = 32 * 128;
+constexpr size_t kPairSmemBytesStaged = kPairSmemBytes + 4 * 2 * kPairOutBytes;
 
 enum : unsigned int {
   kSitePairProducer = 0x311,
@@ -286,15 +298,21 @@ enum : unsigned int {
   kSitePairDrain = 0x315,
 };
 
-template <int QT>
+// STORE = 0: each epilogue lane stores its own row of the tile from registers
+// (out type chosen at run time).  STORE = 1: each epilogue warp writes 32 rows
+// x 128 bytes into a swizzled shared-memory buffer (two per warp, alternating)
+// and one lane stores it with a bulk tensor copy (this GPU's own memory; the
+// copy clips rows and columns past the matrix); OB = 1: bf16 out, else fp32.
+template <int QT, int STORE = 0, int OB = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qgemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                      GemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_c, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPairStages * kPairABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint8_t* sOut = sB + kPairStages * kPairBBytes;  // STORE = 1 only
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + (STORE ? 4 * 2 * kPairOutBytes : 0));
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
@@ -342,7 +360,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain below
       for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
         int tm, tn;
-        gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+        gemm_tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
         const int b_row = tn * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -405,6 +423,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
+  } else if (STORE == 1) {
+    const int quad = warp & 3;
+    const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
+    const uint32_t tempty_leader1 = map_to_rank(&tempty[1], 0);
+    constexpr int kChunkCols = OB ? 64 : 32;  // columns per 128-byte row chunk
+    uint8_t* outbuf = sOut + quad * (2 * kPairOutBytes);
+    const uint32_t swz = static_cast<uint32_t>(lane & 7);
+    int nbuf = 0;
+    int lt = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++lt) {
+      int tm, tn;
+      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
+      const uint32_t acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, kSitePairEpilogue);
+      if (bar_or(1, 128, !ok)) break;
+      tc_fence_after();
+      const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quad * 32;  // this warp's 32 rows
+      const int row = row0 + lane;
+      const float sa = row < p.m ? p.sa[row] : 0.f;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256u;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += kChunkCols) {
+        const int col0 = tn * 256 + c0;
+        uint32_t w[32];  // this row's 128 bytes of the chunk
+#pragma unroll
+        for (int hh = 0; hh < (OB ? 2 : 1); ++hh) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + c0 + 32 * hh, r);
+          tmem_ld_wait();
+          reg_fence32(r);
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = (QT == 0) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+            const int col = col0 + 32 * hh + j;
+            const float sb = col < p.n ? __ldg(p.sb + col) : 0.f;
+            y[j] = (a * sa) * sb;
+          }
+          if (OB) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * e], y[2 * e + 1]);
+              w[16 * hh + e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(y[j]);
+          }
+        }
+        uint8_t* buf = outbuf + (nbuf & 1) * kPairOutBytes;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done with it
+        __syncwarp();
+        // Row `lane` at byte lane * 128; its 16-byte unit j at position j ^ (lane % 8)
+        // (the 128-byte swizzle the tensor map describes): conflict-free 16-byte stores.
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((static_cast<uint32_t>(j) ^ swz) << 4)) =
+              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < p.m && col0 < p.n) {
+          tma_store_2d(&tm_c, buf, col0, row0);
+          bulk_commit();
+        }
+        ++nbuf;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+    if (lane == 0) bulk_wait<0>();  // every output store has completed
   } else {
     const int quad = warp & 3;
     const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
@@ -412,7 +503,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int lt = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++lt) {
       int tm, tn;
-      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
       const uint32_t acc = lt & 1;
       const uint32_t acc_phase = (lt >> 1) & 1;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, kSitePairEpilogue);

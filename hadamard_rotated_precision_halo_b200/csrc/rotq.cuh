@@ -1105,6 +1105,286 @@ __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
 }
 
 // ------------------------------------------------------------------------------------------
+// rotq_cols_tm: rotation along dimension 0 (one scale per column, up to 32768
+// rows) with each strip's rotated values parked in tensor memory while the
+// cluster reduces the column maxima.
+//
+// A 32-column strip's 128-row blocks are spread over a cluster of CL CTAs of
+// NW warps, BW blocks per warp.  A warp brings a block in by TMA (two-stage
+// ring, loads two blocks ahead), rotates it in registers (lane layout of
+// cols_load_fwht), writes the fp32 values to its own tensor-memory lanes
+// (tcgen05.st, 128 columns per block) and folds its column maxima into the
+// CTA's partial vector with shared-memory atomics.  The warp that completes the
+// CTA's count for the strip sends the partial vector (128 bytes) to every
+// cluster CTA with st.async, completing bytes on that CTA's mbarrier.  No warp
+// waits for another warp of its CTA.
+//
+// SLOTS = 2: tensor memory holds two strips.  A warp rotates strip k, sends,
+// and only then waits for strip k - 1's maxima (which had the whole rotation
+// of strip k to arrive), reads strip k - 1 back (tcgen05.ld), quantises it and
+// stores its codes by TMA from a code tile of its own.  SLOTS = 1 (taller
+// matrices, two blocks per warp): one strip, quantised after its own maxima.
+//
+// Buffers reused across strips, and why each reuse is safe:
+//   s_red[k % 2], s_cnt[k % 2]  -- a warp contributes to strip k + 2 only after
+//       it has waited for strip k's maxima, which include this CTA's own
+//       strip-k message, sent after the last contributor cleared the buffer.
+//   s_slot[k % 4], red_bar[k % 4] -- a peer sends strip k + 4 only after its
+//       wait for strip k + 2, which needs this CTA's strip-k + 2 message, sent
+//       after every warp here has finished strip k (read its slots; thread 0
+//       re-armed the barrier).
+//   tensor-memory slot k % SLOTS -- written in strip k + SLOTS by the same warp
+//       that read it back (program order, after tcgen05.wait::ld).
+// ------------------------------------------------------------------------------------------
+struct RotqColsTmParams {
+  float* scales;
+  int64_t cols;
+  int strips;   // ceil(cols / 32)
+  int nblocks;  // padded rows / 128
+  float qmax;
+  float scale_mult;  // 1 / (qmax * sqrt(128))
+  RotqExtras ex;     // EXT = 1 only
+};
+
+enum : unsigned int { kSiteRotqColsTmLoad = 0x211, kSiteRotqColsTmReduce = 0x212, kSiteRotqColsTmDrain = 0x213 };
+
+constexpr int kColsTmSlotBufs = 4;
+constexpr int kColsCodeBytes = 128 * kColsStrip;  // one 128 x 32 code tile
+
+// Dynamic shared memory of rotq_cols_tm: per warp two input stages and two
+// code tiles, plus alignment slack.
+constexpr size_t cols_tm_smem(int nw) { return static_cast<size_t>(nw) * (2 * kColsInBytes + 2 * kColsCodeBytes) + 128; }
+
+template <int NW, int SLOTS, int BW>
+constexpr uint32_t cols_tm_tmem_cols() { return static_cast<uint32_t>(SLOTS * (NW / 4) * BW * 128); }
+
+template <int QT, int NW, int SLOTS, int BW, int EXT = 0>
+__global__ void __launch_bounds__(NW * 32, 1)
+    rotq_cols_tm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                        RotqColsTmParams p) {
+  static_assert(NW % 4 == 0 && (SLOTS == 1 || SLOTS == 2), "warps come in groups of four tensor-memory quadrants");
+  constexpr uint32_t kTmemCols = cols_tm_tmem_cols<NW, SLOTS, BW>();
+  static_assert(kTmemCols == 256 || kTmemCols == 512, "tensor-memory allocation must be a power of two");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t ld_bar[NW][2];                                        // TMA loads, per warp and stage
+  __shared__ uint64_t red_bar[kColsTmSlotBufs];                             // cluster maxima received
+  __shared__ uint32_t s_red[2][kColsStrip];                                 // this CTA's partial maxima
+  __shared__ uint32_t s_cnt[2];                                             // warps done with the strip
+  __shared__ __align__(16) uint32_t s_slot[kColsTmSlotBufs][16][kColsStrip];  // every cluster CTA's maxima
+  __shared__ uint32_t s_tmem;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int pcol = lane & 15;
+  const int h = lane >> 4;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const uint32_t slot_bytes = csize * kColsStrip * 4;
+
+  uint8_t* s_in = smem + warp * (2 * kColsInBytes);
+  uint8_t* s_code = smem + NW * (2 * kColsInBytes) + warp * (2 * kColsCodeBytes);
+
+  if (threadIdx.x < 2 * kColsStrip) (&s_red[0][0])[threadIdx.x] = 0u;
+  if (threadIdx.x < 2) s_cnt[threadIdx.x] = 0u;
+  if (lane == 0) {
+    mbar_init(&ld_bar[warp][0], 1);
+    mbar_init(&ld_bar[warp][1], 1);
+  }
+  if (threadIdx.x == 0)
+    for (int b = 0; b < kColsTmSlotBufs; ++b) mbar_init(&red_bar[b], 1);
+  fence_mbar_init();
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0)
+    for (int b = 0; b < kColsTmSlotBufs; ++b) mbar_arrive_expect_tx(&red_bar[b], slot_bytes);  // strips 0..3
+  cluster_arrive();  // every peer is running and initialised before the first remote store
+  cluster_wait();
+  griddep_wait();
+  // Every CTA has its tensor memory before a dependent grid may launch (whose
+  // CTAs could otherwise hold tensor memory while waiting for this grid).
+  griddep_launch_dependents();
+
+  const uint32_t tmem_base = s_tmem;
+  const uint32_t t_lane = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+  const int wp = warp / 4;
+  const int blk0 = (static_cast<int>(crank) * NW + warp) * BW;  // this warp's first block of every strip
+  const int nvalid = max(0, min(BW, p.nblocks - blk0));
+  const int first = blockIdx.y;
+  const int step = gridDim.y;
+  const int nmine = first < p.strips ? (p.strips - first + step - 1) / step : 0;
+  const int nitems = nmine * nvalid;  // (strip, block) items of this warp, in order
+
+  uint32_t ld_issued = 0, ld_par = 0;
+  auto issue = [&](int i) {
+    const int k = i / nvalid, j = i % nvalid;  // called only when nvalid > 0
+    const int st = i & 1;
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(i >> 1));
+    mbar_arrive_expect_tx(&ld_bar[warp][st], kColsInBytes);
+    tma_load_2d(s_in + st * kColsInBytes, &tm_x, &ld_bar[warp][st], (first + k * step) * kColsStrip,
+                (blk0 + j) * 128);
+  };
+  if (lane == 0) {
+    if (nitems > 0) issue(0);
+    if (nitems > 1) issue(1);
+  }
+
+  bool dead = false;  // a wait ran out: stop waiting, keep sending so that peers do not wait on this CTA
+  int ncodes = 0;     // code tiles written by this warp (they alternate)
+
+  auto rotate_strip = [&](int k) {
+    const int par = k & 1;
+    float m0 = 0.f, m1 = 0.f;
+    for (int j = 0; j < nvalid; ++j) {
+      const int i = k * nvalid + j;
+      const int st = i & 1;
+      float2 v[64];
+      if (!dead) {
+        const bool ok = mbar_wait(&ld_bar[warp][st], (i >> 1) & 1, kSiteRotqColsTmLoad);
+        dead = __any_sync(0xffffffffu, !ok);
+      }
+      if (!dead) {
+        cols_load_fwht<EXT>(reinterpret_cast<const uint32_t*>(s_in + st * kColsInBytes), pcol, h, v,
+                            EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(blk0 + j) * 128 : nullptr);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) v[q] = make_float2(0.f, 0.f);
+      }
+      __syncwarp();  // every lane has read the stage
+      if (lane == 0 && !dead && i + 2 < nitems) issue(i + 2);
+      cols_fwht_rest(v);
+      const float2 mm = absmax64_cols(v);
+      m0 = fmaxf(m0, mm.x);
+      m1 = fmaxf(m1, mm.y);
+      const uint32_t col = static_cast<uint32_t>((((SLOTS == 2 ? par : 0) * (NW / 4) + wp) * BW + j) * 128);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          r[2 * e] = __float_as_uint(v[16 * q + e].x);
+          r[2 * e + 1] = __float_as_uint(v[16 * q + e].y);
+        }
+        tmem_st_32x32b_x32(tmem_base + t_lane + col + 32 * q, r);
+      }
+    }
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
+    if (h == 0 && nvalid > 0) {
+      atomicMax(&s_red[par][2 * pcol], __float_as_uint(m0));
+      atomicMax(&s_red[par][2 * pcol + 1], __float_as_uint(m1));
+    }
+    __syncwarp();
+    uint32_t last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&s_cnt[par], 1u) == static_cast<uint32_t>(NW - 1) ? 1u : 0u;
+      if (last) __threadfence_block();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __syncwarp();
+      // Lane (c, r0): 16-byte chunk c = lane & 7 of the 32 maxima, to cluster
+      // ranks r0 = lane >> 3, r0 + 4, ...
+      const int c = lane & 7;
+      const volatile uint32_t* sr = &s_red[par][4 * c];
+      const uint4 vec = make_uint4(sr[0], sr[1], sr[2], sr[3]);
+      __syncwarp();  // every lane has read the vector before it is cleared for strip k + 2
+      if (lane < 8) *reinterpret_cast<uint4*>(&s_red[par][4 * lane]) = make_uint4(0u, 0u, 0u, 0u);
+      if (lane == 0) s_cnt[par] = 0u;
+      __syncwarp();
+      const int b4 = k & (kColsTmSlotBufs - 1);
+      for (uint32_t r = static_cast<uint32_t>(lane >> 3); r < csize; r += 4)
+        st_async_v4(map_to_rank(&s_slot[b4][crank][4 * c], r), vec, map_to_rank(&red_bar[b4], r));
+    }
+  };
+
+  auto quantise_strip = [&](int k) {
+    const int b4 = k & (kColsTmSlotBufs - 1);
+    if (!dead) {
+      const bool ok = mbar_wait_cluster(&red_bar[b4], (k >> 2) & 1, kSiteRotqColsTmReduce);
+      dead = __any_sync(0xffffffffu, !ok);
+    }
+    uint32_t u0 = 0u, u1 = 0u;
+    for (uint32_t r = 0; r < csize; ++r) {
+      const uint2 pr = *reinterpret_cast<const uint2*>(&s_slot[b4][r][2 * pcol]);
+      u0 = max(u0, pr.x);
+      u1 = max(u1, pr.y);
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&red_bar[b4], slot_bytes);  // armed for strip k + 4
+    const float cm0 = __uint_as_float(u0), cm1 = __uint_as_float(u1);
+    const float r0 = cm0 > 0.f ? __fdiv_rn(p.qmax, cm0) : 0.f;
+    const float r1 = cm1 > 0.f ? __fdiv_rn(p.qmax, cm1) : 0.f;
+    const int c0 = (first + k * step) * kColsStrip;
+    if (crank == 0 && warp == 0 && h == 0) {
+      if (c0 + 2 * pcol < p.cols) p.scales[c0 + 2 * pcol] = cm0 * p.scale_mult;
+      if (c0 + 2 * pcol + 1 < p.cols) p.scales[c0 + 2 * pcol + 1] = cm1 * p.scale_mult;
+    }
+    if (nvalid > 0) tmem_st_wait();  // this warp's stores of the strip have landed
+    for (int j = 0; j < nvalid; ++j) {
+      const uint32_t col = static_cast<uint32_t>((((SLOTS == 2 ? (k & 1) : 0) * (NW / 4) + wp) * BW + j) * 128);
+      // The block's 128 columns in four loads and one wait (one round trip).
+      uint32_t r[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld_32x32b_x32(tmem_base + t_lane + col + 32 * q, r[q]);
+      tmem_ld_wait();
+      float2 v[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        reg_fence32(r[q]);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          v[16 * q + e] = make_float2(__uint_as_float(r[q][2 * e]), __uint_as_float(r[q][2 * e + 1]));
+      }
+      uint8_t* tile = s_code + (ncodes & 1) * kColsCodeBytes;
+      if (lane == 0) bulk_wait_read<1>();  // the store that last read this tile is done with it
+      __syncwarp();
+      {
+        const bool col_ok = c0 + 2 * pcol < p.cols;
+        const uint16_t* rnd = EXT && p.ex.rand && col_ok
+                                  ? p.ex.rand + static_cast<int64_t>(blk0 + j) * 128 * p.ex.ld_rand + c0 + 2 * pcol
+                                  : nullptr;
+        cols_write_codes<QT, EXT>(tile, v, r0, r1, pcol, h, rnd, p.ex.ld_rand);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tm_q, tile, c0, (blk0 + j) * 128);
+        bulk_commit();
+      }
+      ++ncodes;
+    }
+  };
+
+  for (int k = 0; k < nmine; ++k) {
+    rotate_strip(k);
+    if (SLOTS == 2) {
+      if (k >= 1) quantise_strip(k - 1);
+    } else {
+      quantise_strip(k);
+    }
+  }
+  if (SLOTS == 2 && nmine >= 1) quantise_strip(nmine - 1);
+
+  if (lane == 0) {
+    drain_loads(ld_bar[warp], 2, ld_issued, ld_par, kSiteRotqColsTmDrain);
+    bulk_wait<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, kTmemCols);
+  cluster_arrive();  // no CTA leaves while a peer could still store into its shared memory
+  cluster_wait();
+}
+
+// ------------------------------------------------------------------------------------------
 // rotq_cols_grouped: rotation along dimension 0 with group-wise scales, one per
 // `group` (64 or 128) consecutive rows of a column.  A group never leaves a
 // 128-row block, so every warp works alone: persistent warps walk the (block,
@@ -1252,6 +1532,135 @@ __global__ void __launch_bounds__(128, 3)
   }
   if (lane == 0) {
     drain_loads(bars[warp], 2, ld_issued, ld_par, kSiteRotqColsGrDrain);
+    bulk_wait<0>();
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// rotq_cols_split: the dimension-0 rotation split at the column maxima, for a
+// matrix whose rows are spread over several devices (each holds whole 128-row
+// blocks).  MODE 0: the per-column maxima of the unnormalised transform,
+// max |H x| over this device's rows, merged into amax[] with atomicMax (the
+// caller zeroes it; one device's vector is then reduced with the others').
+// MODE 1: codes and scales from given per-column maxima (the maxima over
+// every device's rows): the same rotation, multipliers qmax / amax and codes
+// as the single-device kernels, so the codes are those of the whole matrix.
+// Independent warps over the (128-row block, 32-column strip) items, lane
+// layout of cols_load_fwht, two-stage TMA ring per warp.
+// ------------------------------------------------------------------------------------------
+struct RotqColsSplitParams {
+  float* amax;          // MODE 0: [cols] maxima out (fp32 bits, atomicMax); MODE 1: [cols] maxima in
+  float* scales;        // MODE 1: [cols] scales out (amax * scale_mult)
+  int64_t cols;
+  int strips;           // ceil(cols / 32)
+  int nblocks;          // rows_p / 128
+  float qmax;
+  float scale_mult;     // 1 / (qmax * sqrt(128))
+};
+
+enum : unsigned int { kSiteRotqColsSplitLoad = 0x221, kSiteRotqColsSplitDrain = 0x222 };
+
+template <int QT, int MODE>
+__global__ void __launch_bounds__(128, 3)
+    rotq_cols_split_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+                           RotqColsSplitParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t bars[4][2];
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int pcol = lane & 15;
+  const int h = lane >> 4;
+  uint8_t* s_in = smem + warp * (2 * kColsInBytes);
+
+  if (lane == 0) {
+    mbar_init(&bars[warp][0], 1);
+    mbar_init(&bars[warp][1], 1);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const int64_t items = static_cast<int64_t>(p.nblocks) * p.strips;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * 4;
+  const int64_t nmine = wid < items ? (items - wid + nw - 1) / nw : 0;
+
+  uint32_t ld_issued = 0, ld_par = 0;
+  auto issue = [&](int64_t k) {
+    const int64_t it = wid + k * nw;
+    const int b = static_cast<int>(it / p.strips), sidx = static_cast<int>(it % p.strips);
+    const int st = static_cast<int>(k & 1);
+    note_load(ld_issued, ld_par, st, static_cast<uint32_t>(k >> 1));
+    mbar_arrive_expect_tx(&bars[warp][st], kColsInBytes);
+    tma_load_2d(s_in + st * kColsInBytes, &tm_x, &bars[warp][st], sidx * kColsStrip, b * 128);
+  };
+  if (lane == 0) {
+    if (nmine > 0) issue(0);
+    if (nmine > 1) issue(1);
+  }
+
+  bool dead = false;
+  for (int64_t k = 0; k < nmine; ++k) {
+    const int par = static_cast<int>(k & 1);
+    const int64_t it = wid + k * nw;
+    const int b = static_cast<int>(it / p.strips);
+    const int c0 = static_cast<int>(it % p.strips) * kColsStrip;
+    const int col = c0 + 2 * pcol;
+    float2 v[64];
+    if (!dead) {
+      const bool ok = mbar_wait(&bars[warp][par], static_cast<uint32_t>((k >> 1) & 1), kSiteRotqColsSplitLoad);
+      dead = __any_sync(0xffffffffu, !ok);
+    }
+    if (!dead) {
+      cols_load_fwht<0>(reinterpret_cast<const uint32_t*>(s_in + par * kColsInBytes), pcol, h, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = make_float2(0.f, 0.f);
+    }
+    __syncwarp();
+    if (MODE == 0) {
+      // The stage is free once read: refill it with item k + 2 now.
+      if (lane == 0 && !dead && k + 2 < nmine) issue(k + 2);
+      cols_fwht_rest(v);
+      const float2 mm = absmax64_cols(v);
+      const float m0 = fmaxf(mm.x, __shfl_xor_sync(0xffffffffu, mm.x, 16));
+      const float m1 = fmaxf(mm.y, __shfl_xor_sync(0xffffffffu, mm.y, 16));
+      if (h == 0) {
+        unsigned int* am = reinterpret_cast<unsigned int*>(p.amax);
+        if (col < p.cols) atomicMax(am + col, __float_as_uint(m0));
+        if (col + 1 < p.cols) atomicMax(am + col + 1, __float_as_uint(m1));
+      }
+    } else {
+      cols_fwht_rest(v);
+      // The other stage held item k - 1, whose codes were stored from it at
+      // the end of the previous iteration: once that store has read them, refill it.
+      if (lane == 0 && !dead && k >= 1 && k + 1 < nmine) {
+        bulk_wait_read<0>();
+        issue(k + 1);
+      }
+      const float cm0 = col < p.cols ? __ldg(p.amax + col) : 0.f;
+      const float cm1 = col + 1 < p.cols ? __ldg(p.amax + col + 1) : 0.f;
+      const float r0 = cm0 > 0.f ? __fdiv_rn(p.qmax, cm0) : 0.f;
+      const float r1 = cm1 > 0.f ? __fdiv_rn(p.qmax, cm1) : 0.f;
+      if (b == 0 && h == 0) {
+        if (col < p.cols) p.scales[col] = cm0 * p.scale_mult;
+        if (col + 1 < p.cols) p.scales[col + 1] = cm1 * p.scale_mult;
+      }
+      uint8_t* s_codes = s_in + par * kColsInBytes;  // every lane has read this stage (warp sync above)
+      cols_write_codes<QT>(s_codes, v, r0, r1, pcol, h);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tm_q, s_codes, c0, b * 128);
+        bulk_commit();
+      }
+    }
+  }
+  if (lane == 0) {
+    drain_loads(bars[warp], 2, ld_issued, ld_par, kSiteRotqColsSplitDrain);
     bulk_wait<0>();
   }
 }

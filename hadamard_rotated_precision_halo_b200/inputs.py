@@ -111,6 +111,8 @@ LLAMA7B_FFN_DOWN = LayerShapes(tokens=8192, hidden=4096, ffn=11008, kv=4096,
                                gemms=[Gemm("down", 8192, 4096, 11008, "mlp_act")])
 # One GEMM of the Llama-70B layer: the gate projection (X[4096,8192], W[28672,8192]).
 LLAMA70B_GATE = LayerShapes(gemms=[Gemm("gate", 4096, 28672, 8192, "mlp_in")])
+# Another: the query projection (X[4096,8192], W[8192,8192]).
+LLAMA70B_Q = LayerShapes(gemms=[Gemm("q", 4096, 8192, 8192, "attn_in")])
 
 
 def layer_inputs(shapes: LayerShapes, seed: int, device) -> dict:

@@ -150,6 +150,56 @@ halo_status_t halo_hadamard_quantize_dual(const void* x_bf16, int64_t rows, int6
                                           void* q_e4m3, int64_t ld_qf8, float* scales_e4m3, void* stream);
 
 /*
+ * Both code sets of one matrix that feeds two GEMMs of the backward pass
+ * (dY: dX = dY W contracts its columns, dW = dY^T X its rows): rotated along
+ * the contiguous dimension (blocks of blk, one scale per row) into q_rows /
+ * scales_rows, exactly as halo_hadamard_quantize(axis HALO_AXIS_COLS), and
+ * along dimension 0 (blocks of 128, one scale per column) into q_cols /
+ * scales_cols, exactly as halo_hadamard_quantize(axis HALO_AXIS_ROWS).  The
+ * two rotations run back to back on the stream, so that the second reads X
+ * from L2 when X fits there (up to about 64 MB): one read of X from memory
+ * for both code sets.  Arguments, layouts and errors as the two calls; both
+ * are checked before either is launched.  Defined by: HALO paper page,
+ * abstract (rotations in the backward pass: dY is rotated along N for dX and
+ * along the tokens for dW).
+ */
+halo_status_t halo_hadamard_quantize_both(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                                          int blk, int qtype, void* q_rows, int64_t ld_qr,
+                                          float* scales_rows, void* q_cols, int64_t ld_qc,
+                                          float* scales_cols, void* stream);
+
+/*
+ * The dimension-0 rotation split at its column maxima, for a matrix whose
+ * rows are spread over several devices, each holding whole 128-row blocks
+ * (fully sharded data parallelism with low-precision communication: HALO
+ * paper page, "technical framework").  The devices exchange one fp32 vector
+ * of column maxima instead of the bf16 rows.
+ *
+ * halo_hadamard_colmax: amax_out[c] = the largest |u| over this device's rows
+ *   of column c, u = H_128 x the unnormalised block transform along dimension 0
+ *   (rows zero-padded to whole blocks as in halo_hadamard_quantize).  The
+ *   caller merges the devices' vectors by element-wise maximum (an all-reduce).
+ *   amax_out: [cols] fp32, device memory, 16-byte aligned, overwritten (the
+ *   call clears it on the stream, then accumulates).
+ * halo_hadamard_quantize_colmax: codes and scales of X[rows, cols] rotated
+ *   along dimension 0 with given column maxima amax[c] (those of every
+ *   device's rows): q = round_half_even(u * qmax / amax[c]) clamped to +-127
+ *   (INT8), or the E4M3 encoding of u * qmax / amax[c] (satfinite);
+ *   scales_out[c] = amax[c] / (qmax sqrt(128)); amax[c] = 0 gives code 0 and
+ *   scale 0.  Given the maxima of the whole matrix, each device's codes and
+ *   scales are byte for byte those halo_hadamard_quantize (axis
+ *   HALO_AXIS_ROWS) writes for its rows of the whole matrix.
+ * blk must be 128 and cols % 8 == 0; x, q_out, ld_q, scales_out, layouts and
+ * errors as halo_hadamard_quantize with axis HALO_AXIS_ROWS; amax: [cols]
+ * fp32, device, 16-byte aligned, not written.
+ */
+halo_status_t halo_hadamard_colmax(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x, int blk,
+                                   float* amax_out, void* stream);
+halo_status_t halo_hadamard_quantize_colmax(const void* x_bf16, int64_t rows, int64_t cols,
+                                            int64_t ld_x, int blk, int qtype, const float* amax,
+                                            void* q_out, int64_t ld_q, float* scales_out, void* stream);
+
+/*
  * Low-precision GEMM on codes with a dequantising epilogue:
  *     C[i, j] = (sum_k A[i, k] B[j, k]) * s_a[i] * s_b[j]
  * A is M x K and B is N x K (logically).  a_major / b_major give their

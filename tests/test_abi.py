@@ -151,6 +151,23 @@ def test_linear_fwd_noalloc_host_validation(lib):
     assert f(FAKE, FAKE, 8192, 8192, 4096, 128, 0, FAKE, 0, None) == WORKSPACE  # beyond the static scratch
 
 
+def test_split_dim0_host_validation(lib):
+    c = lib.halo_hadamard_colmax
+    assert c(None, 256, 64, 64, 128, FAKE, None) == NULL
+    assert c(FAKE, 256, 64, 64, 128, None, None) == NULL
+    assert c(FAKE, 256, 64, 64, 256, FAKE, None) == BLOCK       # dimension 0 takes 128-blocks only
+    assert c(FAKE, 256, 60, 64, 128, FAKE, None) == SHAPE       # cols % 8
+    assert c(FAKE, 256, 64, 60, 128, FAKE, None) == SHAPE       # ld_x < cols
+    assert c(MISALIGNED, 256, 64, 64, 128, FAKE, None) == ALIGN
+    assert c(FAKE, 256, 64, 64, 128, MISALIGNED, None) == ALIGN
+    q = lib.halo_hadamard_quantize_colmax
+    assert q(FAKE, 256, 64, 64, 128, 0, None, FAKE, 64, FAKE, None) == NULL
+    assert q(FAKE, 256, 64, 64, 128, 0, FAKE, None, 64, FAKE, None) == NULL
+    assert q(FAKE, 256, 64, 64, 128, 7, FAKE, FAKE, 64, FAKE, None) == DTYPE
+    assert q(FAKE, 256, 64, 64, 128, 0, MISALIGNED, FAKE, 64, FAKE, None) == ALIGN
+    assert q(FAKE, 256, 64, 64, 128, 0, FAKE, FAKE, 72, FAKE, None) == ALIGN  # ld_q % 16
+
+
 def test_hadamard_quantize_ex_host_validation(lib):
     f = lib.halo_hadamard_quantize_ex
     # plain arguments are checked as for halo_hadamard_quantize

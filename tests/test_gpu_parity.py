@@ -54,7 +54,11 @@ def test_rotq_rows_parity(qtype, rows, cols, blk):
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
 @pytest.mark.parametrize("rows,cols", [(1024, 208), (384, 96), (2048, 64), (128, 16), (4096, 48), (1152, 48),
-                                       (8320, 32), (28672, 64)])
+                                       (8320, 32), (28672, 64),
+                                       # clusters of 16 CTAs (128 and 256 blocks of 128 rows)
+                                       (16384, 96), (32768, 64),
+                                       # several strips per cluster: every reused buffer goes round
+                                       (4096, 8192), (16384, 1056), (28672, 1024)])
 def test_rotq_cols_parity(qtype, rows, cols):
     x = inputs.activations(rows, cols, seed=rows + 3 * cols, device="cpu")
     x[:, min(5, cols - 1)] = 0  # an all-zero column
@@ -590,3 +594,39 @@ def test_rotq_rows_longest_row(qtype):
     torch.cuda.synchronize()
     codes, scales, t = oracle_operand(x, 1, 128, qtype)
     check_codes(q, s, codes, scales, t, qtype, blk=128, axis=1)
+
+
+# ------------------------------------------------------- dY's two code sets from one read
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("rows,cols", [(4096, 1024), (1000, 520), (256, 8192)])
+def test_rotq_both_axes_parity(qtype, rows, cols):
+    """halo_hadamard_quantize_both: the per-row codes (rotation along the
+    contiguous dim) and the per-column codes (along dim 0) of one matrix, byte
+    for byte those of the two separate calls, and both against the oracle."""
+    x = inputs.grads(rows, cols, seed=rows + cols, device="cpu")
+    x[:, 1] = 0  # an all-zero column
+    xd = _cuda(x)
+    qr, sr, qc, sc = halo.halo_hadamard_quantize_both(xd, 128, qtype)
+    q1, s1 = halo.halo_hadamard_quantize(xd, COLS, 128, qtype)
+    q0, s0 = halo.halo_hadamard_quantize(xd, ROWS, 128, qtype)
+    torch.cuda.synchronize()
+    assert torch.equal(qr.view(torch.uint8), q1.view(torch.uint8)) and torch.equal(sr, s1)
+    assert torch.equal(qc.view(torch.uint8), q0.view(torch.uint8)) and torch.equal(sc, s0)
+    codes, scales, t = oracle_operand(x, 1, 128, qtype)
+    check_codes(qr, sr, codes, scales, t, qtype, blk=128, axis=1)
+    codes, scales, t = oracle_operand(x, 0, 128, qtype)
+    check_codes(qc, sc, codes, scales, t, qtype, blk=128, axis=0)
+
+
+@pytest.mark.parametrize("axis,rows,cols", [(ROWS, 4096, 1024), (ROWS, 16384, 96), (ROWS, 28672, 64)])
+def test_dim0_variants_on_every_kernel_shape(axis, rows, cols):
+    """Random signs and stochastic rounding along dim 0 at the heights that
+    select each dimension-0 kernel configuration."""
+    x = inputs.activations(rows, cols, seed=rows + cols + 7, device="cpu")
+    s = _signs_t(rows, seed=rows + 1)
+    rb = _rand_bits(rows, cols, seed=cols + 3)
+    q, sc = halo.halo_hadamard_quantize_ex(_cuda(x), axis, 128, INT8, signs=_cuda(s), rand_bits=_cuda(rb))
+    torch.cuda.synchronize()
+    v = oracle.rotate_signed(x, 128, 0, s.numpy())
+    codes, scales, t = oracle.quantize_stochastic(v, 1, INT8, rb.numpy())
+    check_codes_stochastic(q, sc, codes, scales, t, rb.numpy(), INT8, blk=128, axis=0)

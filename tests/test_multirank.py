@@ -38,7 +38,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_rank_timing_is_the_max_and_value_counts_all_ranks():
     world = 2
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()  # no fork of a process that may hold a CUDA context
     out = manager.dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     assert out[0] == out[1]
