@@ -118,22 +118,20 @@ Cols1Kernel cols_1pass_kernel(int qtype, int nw, bool ext) {
   return ext ? cols_1pass_for<1, 1>(nw) : cols_1pass_for<1, 0>(nw);
 }
 
-// Dimension-0 rotation with the rotated values parked in tensor memory:
-// variant 0 (<= 64 blocks of 128 rows): 4 warps, two strips in tensor memory;
-// variant 1 (<= 128 blocks): 8 warps, two strips; variant 2 (<= 256 blocks):
-// 8 warps of two blocks each, one strip.
+// Dimension-0 rotation with the rotated values parked in tensor memory, one
+// 8-warp CTA per SM (all of its tensor memory), clusters of as few CTAs as
+// the column needs so that clusters pack the GPCs' SMs:
+// variant 0 (<= 128 blocks of 128 rows): one block per warp, two strips in
+// tensor memory (cluster = blocks / 8); variant 1 (<= 256 blocks): two blocks
+// per warp, one strip (cluster = blocks / 16).
 typedef void (*ColsTmKernel)(const CUtensorMap, const CUtensorMap, RotqColsTmParams);
-constexpr int kColsTmVariants = 3;
-constexpr int kColsTmWarps[kColsTmVariants] = {4, 8, 8};
-constexpr int kColsTmBlocksPerCta[kColsTmVariants] = {4, 8, 16};
+constexpr int kColsTmVariants = 2;
+constexpr int kColsTmWarps[kColsTmVariants] = {8, 8};
+constexpr int kColsTmBlocksPerCta[kColsTmVariants] = {8, 16};
 
 template <int QT, int EXT>
 ColsTmKernel cols_tm_for(int variant) {
-  switch (variant) {
-    case 0: return rotq_cols_tm_kernel<QT, 4, 2, 1, EXT>;
-    case 1: return rotq_cols_tm_kernel<QT, 8, 2, 1, EXT>;
-    default: return rotq_cols_tm_kernel<QT, 8, 1, 2, EXT>;
-  }
+  return variant == 0 ? rotq_cols_tm_kernel<QT, 8, 2, 1, EXT> : rotq_cols_tm_kernel<QT, 8, 1, 2, EXT>;
 }
 
 // ext: random signs and / or stochastic rounding (RotqExtras).
@@ -226,12 +224,10 @@ halo_status_t device_setup(int* dev_out) {
     }
     HALO_CUDA(set_smem_attr(qgemm_kernel<0>, optin));
     HALO_CUDA(set_smem_attr(qgemm_kernel<1>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 1, 0>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 1, 1>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 1, 0>, optin));
-    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 1, 1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<0, 1>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 0>, optin));
+    HALO_CUDA(set_smem_attr(qgemm_pair_kernel<1, 1>, optin));
   }
   d.ready.store(true, std::memory_order_release);
   return d.supported ? HALO_OK : HALO_ERR_UNSUPPORTED;
@@ -287,21 +283,7 @@ struct Launch {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// EXPERIMENT ONLY (removed before commit): A/B switch for the tensor-memory dim-0 kernel.
-static const bool g_cols_tm_enabled = [] {
-  const char* e = getenv("HALO_COLS_TM");
-  return !(e && e[0] == '0');
-}();
-// EXPERIMENT ONLY (removed before commit): raster group of the pair GEMM.
-static const int g_gemm_group_m = [] {
-  const char* e = getenv("HALO_GEMM_GROUPM");
-  return e && atoi(e) > 0 ? atoi(e) : 16;
-}();
-// EXPERIMENT ONLY (removed before commit): A/B switch for the bulk-store GEMM epilogue.
-static const bool g_gemm_staged = [] {
-  const char* e = getenv("HALO_GEMM_STAGED");
-  return !(e && e[0] == '0');
-}();
+
 
 halo_status_t encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
                      const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle sw) {
@@ -581,17 +563,20 @@ halo_status_t launch_rotq_cols(const void* x, int64_t rows, int64_t cols, int64_
   // Rows past the input (zero padding to whole 128-row blocks) are outside the
   // input tensor map and arrive as zeros; the codes cover the padded rows.
   const int nblocks = static_cast<int>(pad_to(rows, 128) / 128);
-  if (g_cols_tm_enabled) {
-    for (int v = 0; v < kColsTmVariants; ++v)
-      if (nblocks <= 16 * kColsTmBlocksPerCta[v])
-        return launch_rotq_cols_tm(x, rows, cols, ld_x, qtype, q, ld_q, scales, ex, ext, stream, v, nblocks, dev);
-  }
-  // Most warps per CTA (up to 4) with at most 16 CTAs per cluster.
+  // Up to 8192 rows: the single-pass kernel with the strip in registers (most
+  // warps per CTA, up to 4, at most 16 CTAs per cluster).  8193..16384 rows:
+  // the strip parked in tensor memory, which reads the input once where the
+  // register kernel would need two passes.  Taller: two passes.  (Measured on
+  // this pool, isolated: 8192 x 8192 69.6 us in registers against 71.7 us in
+  // tensor memory; 16384 x 4096 73.7 us in tensor memory against 84.0 us in
+  // two passes; 28672 x 8192 243.7 us in two passes against 280.6 us.)
   for (int nw = 4; nw >= 1; --nw) {
     if (nblocks % nw == 0 && nblocks / nw <= 16)
       return launch_rotq_cols_1pass(x, rows, cols, ld_x, qtype, q, ld_q, scales, ex, ext, stream, nw, nblocks / nw,
                                     dev);
   }
+  if (nblocks <= 16 * kColsTmBlocksPerCta[0])
+    return launch_rotq_cols_tm(x, rows, cols, ld_x, qtype, q, ld_q, scales, ex, ext, stream, 0, nblocks, dev);
   // Taller matrices: the two-pass kernel (column maxima first, then codes).
   int cl = 8;
   while (cl > 1 && cl > nblocks) cl /= 2;
@@ -830,7 +815,7 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.a_mn = a_mn;
   p.b_mn = b_mn;
-  p.group_m = g_gemm_group_m;
+  p.group_m = kGemmGroupM;
   // Instruction descriptor: D format (bits 4-5), A/B formats (7-9, 10-12),
   // A/B major (15, 16), N >> 3 (17-22), M >> 4 (24-28).
   uint32_t idesc = 0;
@@ -871,13 +856,9 @@ halo_status_t launch_qgemm(const void* a, const float* sa, int a_mn, int64_t ld_
     if (st != HALO_OK) return st;
   }
   typedef void (*PairKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, GemmParams);
-  PairKernel kern;
-  if (g_gemm_staged)
-    kern = qtype == HALO_Q_INT8 ? (bf16_out ? qgemm_pair_kernel<0, 1, 1> : qgemm_pair_kernel<0, 1, 0>)
-                                : (bf16_out ? qgemm_pair_kernel<1, 1, 1> : qgemm_pair_kernel<1, 1, 0>);
-  else
-    kern = qtype == HALO_Q_INT8 ? qgemm_pair_kernel<0> : qgemm_pair_kernel<1>;
-  Launch L(dim3(2 * pairs), dim3(kGemmThreads), g_gemm_staged ? kPairSmemBytesStaged : kPairSmemBytes, stream, 2);
+  const PairKernel kern = qtype == HALO_Q_INT8 ? (bf16_out ? qgemm_pair_kernel<0, 1> : qgemm_pair_kernel<0, 0>)
+                                              : (bf16_out ? qgemm_pair_kernel<1, 1> : qgemm_pair_kernel<1, 0>);
+  Launch L(dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, stream, 2);
   HALO_CUDA(cudaLaunchKernelEx(&L.cfg, kern, tm_a, tm_b, tm_c, p));
   return HALO_OK;
 }

@@ -284,11 +284,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 constexpr int kPairStages = 6;
 constexpr int kPairABytes = 128 * kGemmBK;  // 16 KB: 128 rows of A
 constexpr int kPairBBytes = 128 * kGemmBK;  // 16 KB: 128 N indices of B
-constexpr size_t kPairSmemBytes = kPairStages * (kPairABytes + kPairBBytes) + 1024 + 256;
-// Output staging of the bulk-store epilogue: per epilogue warp two buffers of
-// 32 rows x 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzled.
+// Output staging of the epilogue: per epilogue warp two buffers of 32 rows x
+// 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzled.
 constexpr int kPairOutBytes = 32 * 128;
-constexpr size_t kPairSmemBytesStaged = kPairSmemBytes + 4 * 2 * kPairOutBytes;
+// Dynamic shared memory: stages, output staging, 1 KB alignment slack, barriers.
+constexpr size_t kPairSmemBytes = kPairStages * (kPairABytes + kPairBBytes) + 4 * 2 * kPairOutBytes + 1024 + 256;
 
 enum : unsigned int {
   kSitePairProducer = 0x311,
@@ -298,12 +298,12 @@ enum : unsigned int {
   kSitePairDrain = 0x315,
 };
 
-// STORE = 0: each epilogue lane stores its own row of the tile from registers
-// (out type chosen at run time).  STORE = 1: each epilogue warp writes 32 rows
-// x 128 bytes into a swizzled shared-memory buffer (two per warp, alternating)
-// and one lane stores it with a bulk tensor copy (this GPU's own memory; the
-// copy clips rows and columns past the matrix); OB = 1: bf16 out, else fp32.
-template <int QT, int STORE = 0, int OB = 0>
+// Epilogue: each epilogue warp converts 32 rows x 128 bytes of its accumulator
+// quarter at a time into a swizzled shared-memory buffer (two per warp,
+// alternating) and one lane writes it with a bulk tensor store (this GPU's own
+// memory; the copy clips rows and columns past the matrix), so the stores
+// leave as whole lines and overlap the next chunk.  OB = 1: bf16 out, else fp32.
+template <int QT, int OB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qgemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_c, GemmParams p) {
@@ -311,8 +311,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPairStages * kPairABytes;
-  uint8_t* sOut = sB + kPairStages * kPairBBytes;  // STORE = 1 only
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + (STORE ? 4 * 2 * kPairOutBytes : 0));
+  uint8_t* sOut = sB + kPairStages * kPairBBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + 4 * 2 * kPairOutBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else if (STORE == 1) {
+  } else {
     const int quad = warp & 3;
     const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
     const uint32_t tempty_leader1 = map_to_rank(&tempty[1], 0);
@@ -496,77 +496,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
     }
     if (lane == 0) bulk_wait<0>();  // every output store has completed
-  } else {
-    const int quad = warp & 3;
-    const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
-    const uint32_t tempty_leader1 = map_to_rank(&tempty[1], 0);
-    int lt = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++lt) {
-      int tm, tn;
-      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
-      const uint32_t acc = lt & 1;
-      const uint32_t acc_phase = (lt >> 1) & 1;
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, kSitePairEpilogue);
-      if (bar_or(1, 128, !ok)) break;
-      tc_fence_after();
-      const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
-      const bool row_ok = row < p.m;
-      const float sa = row_ok ? p.sa[row] : 0.f;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256u;
-#pragma unroll 1
-      for (int ch = 0; ch < 256 / 32; ++ch) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(t_row + ch * 32, r);
-        tmem_ld_wait();
-        const int col0 = tn * 256 + ch * 32;
-        if (row_ok && col0 < p.n) {
-          float y[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float a = (QT == 0) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
-            const int col = col0 + j;
-            const float sb = col < p.n ? __ldg(p.sb + col) : 0.f;
-            y[j] = (a * sa) * sb;
-          }
-          const bool full_chunk = col0 + 32 <= p.n;
-          if (p.out_bf16) {
-            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
-            if (full_chunk) {
-              uint4* o4 = reinterpret_cast<uint4*>(out);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[8 * q + 2 * e], y[8 * q + 2 * e + 1]);
-                  w[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                o4[q] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < p.n) out[j] = __float2bfloat16_rn(y[j]);
-            }
-          } else {
-            float* out = static_cast<float*>(p.c) + static_cast<int64_t>(row) * p.ldc + col0;
-            if (full_chunk) {
-              float4* o4 = reinterpret_cast<float4*>(out);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) o4[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < p.n) out[j] = y[j];
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-    }
   }
 
   tc_fence_before();
