@@ -593,15 +593,17 @@ ROTQ_SHAPES = {  # (rows, cols) of every rotate+quantise operand of the 70B laye
 }
 
 
-def measure_rotq_shapes(repeats: int = 10):
+def measure_rotq_shapes(repeats: int = 10, only=None):
     """halo_hadamard_quantize on each shape alone (INT8 and E4M3, block 128), a
     512 MB write between repeats to flush L2; median time and algorithmic GB/s
-    (3 B per element + 4 B per scale)."""
+    (3 B per element + 4 B per scale).  `only` = (direction, (rows, cols)):
+    that one case (both types) and nothing else, e.g. for a profiler."""
     import hadamard_rotated_precision_halo_b200 as halo
 
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     out = []
-    for name, shapes in ROTQ_SHAPES.items():
+    cases = ROTQ_SHAPES if only is None else {only[0]: [only[1]]}
+    for name, shapes in cases.items():
         axis = halo.HALO_AXIS_COLS if name == "along_contiguous_dim" else halo.HALO_AXIS_ROWS
         for r, c in shapes:
             x = inputs.activations(r, c, seed=1, device="cuda")
@@ -622,6 +624,8 @@ def measure_rotq_shapes(repeats: int = 10):
                 out.append({"direction": name, "shape": [r, c], "qtype": "int8" if qt == 0 else "e4m3",
                             "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9})
             del x, q, sc
+    if only is not None:
+        return {"measure": "rotate+quantise per shape", "block": BLK, "results": out}
     # Both encodings from one read (halo_hadamard_quantize_dual): 2 B in + 1 B
     # per code set per element, 4 B per scale of each set.
     for r, c in ROTQ_SHAPES["along_contiguous_dim"]:
@@ -853,10 +857,17 @@ def main():
                     help="print 8-bit GEMM burst / sustained throughput (this library and cuBLAS) and exit")
     ap.add_argument("--rotq-shapes", action="store_true",
                     help="print rotate+quantise time per operand shape of the layer and exit")
+    ap.add_argument("--rotq-shape", default=None, metavar="AXIS:RxC",
+                    help="with --rotq-shapes: only this case, AXIS contig or dim0 (e.g. dim0:16384x4096)")
     args = ap.parse_args()
     if args.measure_peaks or args.rotq_shapes:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        print(json.dumps(measure_peaks() if args.measure_peaks else measure_rotq_shapes()), flush=True)
+        only = None
+        if args.rotq_shape:
+            ax, shape = args.rotq_shape.split(":")
+            r, c = (int(v) for v in shape.split("x"))
+            only = ("along_contiguous_dim" if ax == "contig" else "along_dim0", (r, c))
+        print(json.dumps(measure_peaks() if args.measure_peaks else measure_rotq_shapes(only=only)), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

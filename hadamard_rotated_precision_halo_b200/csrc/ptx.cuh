@@ -100,6 +100,12 @@ __device__ __forceinline__ void note_load(uint32_t& issued, uint32_t& parity, in
   parity = (parity & ~(1u << s)) | ((par & 1u) << s);
 }
 
+// Bring the line holding `p` into L2 ahead of a later load (no register is
+// written, nothing waits).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 // ------------------------------------------------- programmatic dependent launch
 // Wait until the preceding kernel in the stream has completed and its memory is
 // visible (returns at once when the launch has no programmatic dependency).

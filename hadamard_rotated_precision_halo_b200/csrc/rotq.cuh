@@ -334,6 +334,13 @@ __global__ void __launch_bounds__(BLK == 128 && EXT == 0 && QT != kQtDual ? 384 
     const int st = static_cast<int>(it & 1);
     const int par = static_cast<int>(it & 1);
     const int64_t row = first + it * step;
+    if (EXT && p.ex.rand != nullptr && is_active) {
+      // This chunk's random bits (two 128-byte lines) into L2 while the row
+      // is rotated: the code loop below reads them.
+      const uint16_t* rl = p.ex.rand + row * p.ex.ld_rand + static_cast<int64_t>(chunk) * 128;
+      prefetch_l2(rl);
+      prefetch_l2(rl + 64);
+    }
     if (!dead) {
       const bool ok = mbar_wait(&full_bar[grp][st], static_cast<uint32_t>((it >> 1) & 1), kSiteRotqRowsLoad);
       dead = !ok;
@@ -768,6 +775,16 @@ __device__ __forceinline__ void cols_write_codes16(uint8_t* tile, const float2* 
   }
 }
 
+// Stochastic rounding along dimension 0: the random bits of one 128-row block
+// of a 32-column strip (128 lines of 64 bytes, 4 per lane) into L2 ahead of
+// cols_write_codes, whose loads would otherwise wait on memory.
+__device__ __forceinline__ void prefetch_block_rand(const uint16_t* rand, int64_t ld_rand, int64_t row0, int c0,
+                                                    int64_t cols, int lane) {
+  if (rand == nullptr || c0 >= cols) return;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) prefetch_l2(rand + (row0 + 4 * lane + j) * ld_rand + c0);
+}
+
 // Codes of all of the lane's 64 rows x 2 columns.
 template <int QT, int EXT = 0>
 __device__ __forceinline__ void cols_write_codes(uint8_t* tile, const float2 (&v)[64], float r0, float r1, int pcol,
@@ -903,6 +920,7 @@ __global__ void __launch_bounds__(128, EXT ? 2 : 3)
     const uint32_t* blkw = reinterpret_cast<const uint32_t*>(s_in + s * kColsInBytes);
     float2 v[64];
     const int bq = first + step * (2 * nmine - 1 - j);
+    if (EXT) prefetch_block_rand(p.ex.rand, p.ex.ld_rand, static_cast<int64_t>(bq) * 128, c0, p.cols, lane);
     cols_load_fwht<EXT>(blkw, pcol, h, v, EXT && p.ex.signs ? p.ex.signs + static_cast<int64_t>(bq) * 128 : nullptr);
     __syncwarp();
     cols_fwht_rest(v);
@@ -1026,6 +1044,7 @@ __global__ void __launch_bounds__(NW * 32, EXT ? 8 / NW : 12 / NW)
   for (int k = 0; k < nmine; ++k) {
     const int c0 = (first + k * step) * kColsStrip;
     const int par = k & 1;
+    if (EXT) prefetch_block_rand(p.ex.rand, p.ex.ld_rand, static_cast<int64_t>(blk) * 128, c0, p.cols, lane);
     float2 v[64];
     if (!dead) {
       const bool ok = mbar_wait(&bars[warp][par], (k >> 1) & 1, kSiteRotqCols1Load);
@@ -1243,6 +1262,9 @@ __global__ void __launch_bounds__(NW * 32, 1)
     for (int j = 0; j < nvalid; ++j) {
       const int i = k * nvalid + j;
       const int st = i & 1;
+      if (EXT)
+        prefetch_block_rand(p.ex.rand, p.ex.ld_rand, static_cast<int64_t>(blk0 + j) * 128,
+                            (first + k * step) * kColsStrip, p.cols, lane);
       float2 v[64];
       if (!dead) {
         const bool ok = mbar_wait(&ld_bar[warp][st], (i >> 1) & 1, kSiteRotqColsTmLoad);
