@@ -193,6 +193,21 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------ small asynchronous copies
+// 4 bytes from global to shared memory without passing through registers.
+// src_bytes 0 writes zeros and reads nothing (src must still be a valid
+// address).  Copies of one thread are grouped by cp_async_commit(); after
+// cp_async_wait_all() they are visible to that thread, and to the rest of the
+// CTA after a barrier.
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -19,10 +19,12 @@
 //               running sums in registers.  Per group it reads its slice of the
 //               partial (tcgen05.ld), converts it (INT8: exact int32 -> fp32,
 //               |partial| <= 127^2 * 128 < 2^24), multiplies by s_a[i, G] *
-//               s_b[j, G] and adds, then frees the partial.  The s_b of 16
-//               groups are staged in shared memory at a time, so the promotion
-//               warps meet at a barrier once per 16 groups.  The promotion costs a few CUDA-core instructions per
-//               element per group, so it needs many warps to hide its latencies;
+//               s_b[j, G] and adds, then frees the partial.  The s_a and s_b
+//               of 16 groups are staged in shared memory at a time by
+//               asynchronous copies issued one chunk ahead, so the promotion
+//               warps meet at a barrier once per 16 groups and never wait on a
+//               global load.  The promotion costs a few CUDA-core instructions
+//               per element per group, so it needs many warps to hide its latencies;
 //               the four partials let the MMAs run up to three groups ahead.
 // After the last group the running sums are stored as fp32 or bf16.
 #pragma once
@@ -55,9 +57,9 @@ constexpr int kGgThreads = 64 + 32 * kGgPromWarps;  // producer, MMA, promotion
 constexpr int kGgPromThreads = 32 * kGgPromWarps;
 constexpr int kGgColsPerThread = kGgBN * 4 / kGgPromWarps;  // columns of a tile row per promotion thread
 constexpr int kGgChunk = 16;  // groups whose s_b are staged together
-// Dynamic shared memory: stages + 1 KB alignment slack + s_b staging (2 x
-// kGgChunk x 128 floats) + barriers.
-constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 2 * kGgChunk * kGgBN * 4 + 256;
+// Dynamic shared memory: stages + 1 KB alignment slack + scale staging (s_b
+// and s_a, 2 buffers x kGgChunk groups x 128 floats each) + barriers.
+constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 2 * 2 * kGgChunk * kGgBN * 4 + 256;
 
 struct GroupedGemmParams {
   int m, n, k, group;
@@ -82,8 +84,8 @@ __global__ void __launch_bounds__(kGgThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGgStages * kGgABytes;
-  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // [2][kGgChunk][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * kGgChunk * kGgBN);
+  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // s_b, s_a: [2][kGgChunk][128] each
+  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * 2 * kGgChunk * kGgBN);
   uint64_t* empty = full + kGgStages;
   uint64_t* pfull = empty + kGgStages;
   uint64_t* pempty = pfull + kGgPartials;
@@ -193,47 +195,64 @@ __global__ void __launch_bounds__(kGgThreads, 1)
     const int slice = (warp - 2) >> 2;  // this thread's kGgColsPerThread-column slice
     const int row_in_tile = quad * 32 + lane;
     const int ngroups = p.k / p.group;
-    // s_b staging: the 128 threads of the first four promotion warps each load
-    // one column's scale per group into shared memory.
+    // Scale staging: the 128 threads of the first four promotion warps copy,
+    // for a chunk of kGgChunk groups, one column's s_b and one row's s_a per
+    // group into shared memory (warps 2-5 cover lane quarters 2, 3, 0, 1, so
+    // their rows are the tile's 128 rows).  The copies of the next chunk are
+    // issued as soon as a chunk starts and land while it is promoted.
     const bool stager = (warp - 2) < 4;
     const int scol_in_tile = (warp - 2) * 32 + lane;  // valid for stagers: 0..127
+    float* const sb_bufs = sbuf;                              // [2][kGgChunk][128]
+    float* const sa_bufs = sbuf + 2 * kGgChunk * kGgBN;       // [2][kGgChunk][128]
+    auto stage_chunk = [&](int tile, int g0, uint32_t buf) {
+      int tm, tn;
+      gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+      const int gn = min(kGgChunk, ngroups - g0);
+      const int scol = tn * kGgBN + scol_in_tile;
+      const int srow = tm * kGgBM + row_in_tile;
+      const bool cok = scol < p.n, rok = srow < p.m;
+      const float* sbp = p.sb + static_cast<int64_t>(cok ? scol : 0) * p.sb_row + static_cast<int64_t>(g0) * p.sb_grp;
+      const float* sap = p.sa + static_cast<int64_t>(rok ? srow : 0) * p.sa_row + static_cast<int64_t>(g0) * p.sa_grp;
+      float* db = sb_bufs + buf * (kGgChunk * kGgBN) + scol_in_tile;
+      float* da = sa_bufs + buf * (kGgChunk * kGgBN) + row_in_tile;
+      for (int gg = 0; gg < gn; ++gg) {
+        cp_async_4(db + gg * kGgBN, sbp + static_cast<int64_t>(gg) * p.sb_grp, cok ? 4u : 0u);
+        cp_async_4(da + gg * kGgBN, sap + static_cast<int64_t>(gg) * p.sa_grp, rok ? 4u : 0u);
+      }
+      cp_async_commit();
+    };
     uint32_t gi = 0;
-    uint32_t ci = 0;  // s_b chunks staged so far (all tiles): picks the staging buffer
+    uint32_t ci = 0;  // chunks started so far (all tiles): picks the staging buffer
     bool dead = false;
+    if (stager && static_cast<int>(blockIdx.x) < p.num_tiles) stage_chunk(blockIdx.x, 0, 0);
     for (int tile = blockIdx.x; tile < p.num_tiles && !dead; tile += gridDim.x) {
       int tm, tn;
       gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
       const int row = tm * kGgBM + row_in_tile;
       const bool row_ok = row < p.m;
-      const int scol = tn * kGgBN + scol_in_tile;
-      const bool scol_ok = stager && scol < p.n;
-      const float* sa_row = p.sa + static_cast<int64_t>(row_ok ? row : 0) * p.sa_row;
-      const float* sb_col = p.sb + static_cast<int64_t>(scol_ok ? scol : 0) * p.sb_row;
-      float sa_next = row_ok ? __ldg(sa_row) : 0.f;
       float run[kGgColsPerThread];
 #pragma unroll
       for (int j = 0; j < kGgColsPerThread; ++j) run[j] = 0.f;
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + slice * kGgColsPerThread;
 #pragma unroll 1
       for (int g0 = 0; g0 < ngroups; g0 += kGgChunk, ++ci) {
-        // Stage the chunk's s_b (kGgChunk groups x 128 columns).  A buffer is
-        // rewritten only after every thread has passed the barrier of the
-        // chunk after the one that last read it (chunks alternate buffers by
-        // the running chunk count, also across tiles).
-        float* sb_chunk = sbuf + (ci & 1u) * (kGgChunk * kGgBN);
-        const int gn = min(kGgChunk, ngroups - g0);
-        if (stager) {
-          for (int gg = 0; gg < gn; ++gg)
-            sb_chunk[gg * kGgBN + scol_in_tile] = scol_ok ? __ldg(sb_col + static_cast<int64_t>(g0 + gg) * p.sb_grp) : 0.f;
-        }
-        // All promotion threads: publishes sb_chunk; a wait that ran out in
-        // the previous chunk stops all.
+        const uint32_t buf = ci & 1u;
+        if (stager) cp_async_wait_all();  // this chunk's copies, issued one chunk ago
+        // All promotion threads: publishes the chunk's scales, and every thread
+        // has finished the previous chunk, whose buffer is refilled next; a
+        // wait that ran out in the previous chunk stops all.
         if (bar_or(1, kGgPromThreads, dead)) { dead = true; break; }
+        if (stager) {
+          int nt = tile, ng0 = g0 + kGgChunk;
+          if (ng0 >= ngroups) { nt = tile + gridDim.x; ng0 = 0; }
+          if (nt < p.num_tiles) stage_chunk(nt, ng0, buf ^ 1u);
+        }
+        const float* sb_chunk = sb_bufs + buf * (kGgChunk * kGgBN);
+        const float* sa_chunk = sa_bufs + buf * (kGgChunk * kGgBN);
+        const int gn = min(kGgChunk, ngroups - g0);
 #pragma unroll 1
         for (int gg = 0; gg < gn; ++gg, ++gi) {
-          const int g = g0 + gg;
-          const float sa = sa_next;
-          if (g + 1 < ngroups) sa_next = row_ok ? __ldg(sa_row + static_cast<int64_t>(g + 1) * p.sa_grp) : 0.f;
+          const float sa = sa_chunk[gg * kGgBN + row_in_tile];
           const uint32_t pb = gi % kGgPartials;
           if (!dead && !mbar_wait(&pfull[pb], (gi / kGgPartials) & 1u, kSiteGgPromote)) dead = true;
           dead = __any_sync(0xffffffffu, dead);
@@ -317,6 +336,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
     }
   }
 
+  if (warp >= 2) cp_async_wait_all();  // no scale copy lands after the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
