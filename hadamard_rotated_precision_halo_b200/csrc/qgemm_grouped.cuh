@@ -160,25 +160,41 @@ __global__ void __launch_bounds__(kGgThreads, 1)
       const uint32_t b_step = p.b_mn ? 32u * 128u : 32u;
       const uint32_t a_lbo = p.a_mn ? static_cast<uint32_t>(kGgBK * 128) : 16u;
       const uint32_t b_lbo = p.b_mn ? static_cast<uint32_t>(kGgBK * 128) : 16u;
+      const uint64_t as4 = a_step >> 4, bs4 = b_step >> 4;  // one K step in descriptor units
+      const uint32_t idesc = p.idesc;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < kblocks && ok; ++kb) {
           if (!mbar_wait(&full[stage], phase, kSiteGgMma)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * kGgABytes);
-          const uint32_t b_base = smem_u32(sB + stage * kGgBBytes);
+          // Descriptors of the stage's first K step.  A K step adds its byte
+          // offset / 16 to the start-address field (shared-memory offsets stay
+          // below 256 KB, so the 14-bit field never carries).  The issue loop
+          // is short: one thread issues every MMA, and its per-group cost
+          // paces the kernel.
+          const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA + stage * kGgABytes), a_lbo, 1024u);
+          const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB + stage * kGgBBytes), b_lbo, 1024u);
           for (int gs = 0; gs < gpb; ++gs, ++gi) {
             const uint32_t pb = gi % kGgPartials;
             if (!mbar_wait(&pempty[pb], ((gi / kGgPartials) & 1u) ^ 1u, kSiteGgPartial)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + pb * 128u;
-            for (int kk = 0; kk < steps_per_group; ++kk) {
-              const int ks = gs * steps_per_group + kk;  // K step (of 32) inside the block
-              const uint64_t adesc = smem_desc_sw128(a_base + ks * a_step, a_lbo, 1024u);
-              const uint64_t bdesc = smem_desc_sw128(b_base + ks * b_step, b_lbo, 1024u);
-              if (QT == 0)
-                mma_i8(d_tmem, adesc, bdesc, p.idesc, kk > 0 ? 1u : 0u);
-              else
-                mma_f8(d_tmem, adesc, bdesc, p.idesc, kk > 0 ? 1u : 0u);
+            const uint64_t ad = adesc0 + ((gs * steps_per_group * a_step) >> 4);
+            const uint64_t bd = bdesc0 + ((gs * steps_per_group * b_step) >> 4);
+            // group 64: two MMAs of K = 32; group 128: four
+            if (QT == 0) {
+              mma_i8(d_tmem, ad, bd, idesc, 0u);
+              mma_i8(d_tmem, ad + as4, bd + bs4, idesc, 1u);
+              if (steps_per_group == 4) {
+                mma_i8(d_tmem, ad + 2 * as4, bd + 2 * bs4, idesc, 1u);
+                mma_i8(d_tmem, ad + 3 * as4, bd + 3 * bs4, idesc, 1u);
+              }
+            } else {
+              mma_f8(d_tmem, ad, bd, idesc, 0u);
+              mma_f8(d_tmem, ad + as4, bd + bs4, idesc, 1u);
+              if (steps_per_group == 4) {
+                mma_f8(d_tmem, ad + 2 * as4, bd + 2 * bs4, idesc, 1u);
+                mma_f8(d_tmem, ad + 3 * as4, bd + 3 * bs4, idesc, 1u);
+              }
             }
             mma_commit(&pfull[pb]);  // this group's partial is complete
           }
@@ -264,6 +280,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_cols + pb * 128u + ch * 32, r);
           tmem_ld_wait();
+          reg_fence32(r);  // no use of r is scheduled above the wait
           if (ch == kGgColsPerThread / 32 - 1) {
             tc_fence_before();
             __syncwarp();
