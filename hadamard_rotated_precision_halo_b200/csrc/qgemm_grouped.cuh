@@ -8,24 +8,29 @@
 // size 64).  A group's partial product cannot be scaled inside the tensor
 // core, so each group is accumulated on its own and promoted:
 //
-//   warp 0      TMA producer: 128 x 128 A and B tiles (K block of 128 codes,
-//               128-byte swizzle) into a 6-stage ring.
+//   warp 0      TMA producer: a 128 x 128 A tile and a 256 x 128 B tile (as
+//               two 128-wide boxes) per K block of 128 codes, 128-byte
+//               swizzle, into a 4-stage ring.
 //   warp 1      tensor-memory allocator and MMA issuer: for every group, the
-//               group's K steps (group / 32 MMAs of 128x128x32) into one of
-//               four 128-column partial accumulators in tensor memory, then a
+//               group's K steps (group / 32 MMAs of 128x256x32) into one of
+//               two 256-column partial accumulators in tensor memory, then a
 //               commit that marks that partial full.
 //   warps 2-9   promotion: eight warps, two per tensor-memory lane quarter;
-//               each thread owns 64 columns of one tile row and keeps their fp32
-//               running sums in registers.  Per group it reads its slice of the
-//               partial (tcgen05.ld), converts it (INT8: exact int32 -> fp32,
-//               |partial| <= 127^2 * 128 < 2^24), multiplies by s_a[i, G] *
-//               s_b[j, G] and adds, then frees the partial.  The s_a and s_b
-//               of 16 groups are staged in shared memory at a time by
-//               asynchronous copies issued one chunk ahead, so the promotion
-//               warps meet at a barrier once per 16 groups and never wait on a
-//               global load.  The promotion costs a few CUDA-core instructions
-//               per element per group, so it needs many warps to hide its latencies;
-//               the four partials let the MMAs run up to three groups ahead.
+//               each thread owns 128 columns of one tile row and keeps their
+//               fp32 running sums in registers.  Per group it reads its slice
+//               of the partial (tcgen05.ld, 4 columns at a time: small loads
+//               leave the registers to the sums), converts it (INT8: exact
+//               int32 -> fp32, |partial| <= 127^2 * 128 < 2^24), multiplies
+//               by s_a[i, G] * s_b[j, G] and adds, and frees the partial once
+//               its last slice is in registers.  The s_a and s_b of 8 groups
+//               are staged in shared memory at a time by asynchronous copies
+//               issued one chunk ahead, so the promotion warps meet at a
+//               barrier once per 8 groups and never wait on a global load.
+// Each group's hand-over (the MMA thread's waits, fences and commits, the
+// promotion warps' wait and release) costs about the same whatever the tile
+// width, so the 256-column tile does twice the tensor work per hand-over of a
+// 128-column one; the price is two partials instead of four (the MMAs run one
+// group ahead of the promotion).
 // After the last group the running sums are stored as fp32 or bf16.
 #pragma once
 
@@ -45,21 +50,24 @@ enum : unsigned int {
 };
 
 constexpr int kGgBM = 128;
-constexpr int kGgBN = 128;
+constexpr int kGgBN = 256;
 constexpr int kGgBK = 128;
-constexpr int kGgStages = 6;
+constexpr int kGgStages = 4;
 constexpr int kGgABytes = kGgBM * kGgBK;  // 16 KB
-constexpr int kGgBBytes = kGgBN * kGgBK;  // 16 KB
-constexpr int kGgPartials = 4;            // 128-column partial accumulators
+constexpr int kGgBBytes = kGgBN * kGgBK;  // 32 KB: two 128-row (K-major) or 128-column (MN-major) boxes
+constexpr int kGgBHalf = kGgBBytes / 2;
+constexpr int kGgPartials = 2;            // 256-column partial accumulators
 constexpr uint32_t kGgTmemCols = 512;
 constexpr int kGgPromWarps = 8;                      // a multiple of 4 (lane quarters)
 constexpr int kGgThreads = 64 + 32 * kGgPromWarps;  // producer, MMA, promotion
 constexpr int kGgPromThreads = 32 * kGgPromWarps;
 constexpr int kGgColsPerThread = kGgBN * 4 / kGgPromWarps;  // columns of a tile row per promotion thread
-constexpr int kGgChunk = 16;  // groups whose s_b are staged together
-// Dynamic shared memory: stages + 1 KB alignment slack + scale staging (s_b
-// and s_a, 2 buffers x kGgChunk groups x 128 floats each) + barriers.
-constexpr size_t kGgSmemBytes = kGgStages * (kGgABytes + kGgBBytes) + 1024 + 2 * 2 * kGgChunk * kGgBN * 4 + 256;
+constexpr int kGgChunk = 8;  // groups whose scales are staged together
+constexpr int kGgLdCols = 4;  // columns per tensor-memory load (registers: 128 sums + 4)
+// Dynamic shared memory: stages + 1 KB alignment slack + scale staging (2
+// buffers x kGgChunk groups x (256 s_b + 128 s_a) floats) + barriers.
+constexpr size_t kGgSmemBytes =
+    kGgStages * (kGgABytes + kGgBBytes) + 1024 + 2 * kGgChunk * (kGgBN + kGgBM) * 4 + 256;
 
 struct GroupedGemmParams {
   int m, n, k, group;
@@ -84,8 +92,8 @@ __global__ void __launch_bounds__(kGgThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGgStages * kGgABytes;
-  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // s_b, s_a: [2][kGgChunk][128] each
-  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * 2 * kGgChunk * kGgBN);
+  float* sbuf = reinterpret_cast<float*>(sB + kGgStages * kGgBBytes);  // s_b [2][kGgChunk][256], s_a [2][kGgChunk][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sbuf + 2 * kGgChunk * (kGgBN + kGgBM));
   uint64_t* empty = full + kGgStages;
   uint64_t* pfull = empty + kGgStages;
   uint64_t* pempty = pfull + kGgPartials;
@@ -140,10 +148,15 @@ __global__ void __launch_bounds__(kGgThreads, 1)
             tma_load_2d(a_dst, &tm_a, &full[stage], tm * kGgBM, kb * kGgBK);
           else
             tma_load_2d(a_dst, &tm_a, &full[stage], kb * kGgBK, tm * kGgBM);
-          if (p.b_mn)
+          // B in two 128-wide boxes (a box row holds at most 128 swizzled
+          // bytes); a box past the matrix reads as zeros.
+          if (p.b_mn) {
             tma_load_2d(b_dst, &tm_b, &full[stage], tn * kGgBN, kb * kGgBK);
-          else
+            tma_load_2d(b_dst + kGgBHalf, &tm_b, &full[stage], tn * kGgBN + 128, kb * kGgBK);
+          } else {
             tma_load_2d(b_dst, &tm_b, &full[stage], kb * kGgBK, tn * kGgBN);
+            tma_load_2d(b_dst + kGgBHalf, &tm_b, &full[stage], kb * kGgBK, tn * kGgBN + 128);
+          }
           if (++stage == kGgStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -177,7 +190,7 @@ __global__ void __launch_bounds__(kGgThreads, 1)
             const uint32_t pb = gi % kGgPartials;
             if (!mbar_wait(&pempty[pb], ((gi / kGgPartials) & 1u) ^ 1u, kSiteGgPartial)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + pb * 128u;
+            const uint32_t d_tmem = tmem_base + pb * static_cast<uint32_t>(kGgBN);
             const uint64_t ad = adesc0 + ((gs * steps_per_group * a_step) >> 4);
             const uint64_t bd = bdesc0 + ((gs * steps_per_group * b_step) >> 4);
             // group 64: two MMAs of K = 32; group 128: four
@@ -216,10 +229,12 @@ __global__ void __launch_bounds__(kGgThreads, 1)
     // group into shared memory (warps 2-5 cover lane quarters 2, 3, 0, 1, so
     // their rows are the tile's 128 rows).  The copies of the next chunk are
     // issued as soon as a chunk starts and land while it is promoted.
-    const bool stager = (warp - 2) < 4;
-    const int scol_in_tile = (warp - 2) * 32 + lane;  // valid for stagers: 0..127
-    float* const sb_bufs = sbuf;                              // [2][kGgChunk][128]
-    float* const sa_bufs = sbuf + 2 * kGgChunk * kGgBN;       // [2][kGgChunk][128]
+    const bool sb_stager = (warp - 2) < kGgBN / 32;  // warps 2-9: one column each
+    const bool sa_stager = (warp - 2) < 4;           // warps 2-5: one row each
+    const bool stager = sb_stager;
+    const int scol_in_tile = (warp - 2) * 32 + lane;  // valid for s_b stagers: 0..255
+    float* const sb_bufs = sbuf;                               // [2][kGgChunk][256]
+    float* const sa_bufs = sbuf + 2 * kGgChunk * kGgBN;        // [2][kGgChunk][128]
     auto stage_chunk = [&](int tile, int g0, uint32_t buf) {
       int tm, tn;
       gemm_tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
@@ -230,11 +245,12 @@ __global__ void __launch_bounds__(kGgThreads, 1)
       const float* sbp = p.sb + static_cast<int64_t>(cok ? scol : 0) * p.sb_row + static_cast<int64_t>(g0) * p.sb_grp;
       const float* sap = p.sa + static_cast<int64_t>(rok ? srow : 0) * p.sa_row + static_cast<int64_t>(g0) * p.sa_grp;
       float* db = sb_bufs + buf * (kGgChunk * kGgBN) + scol_in_tile;
-      float* da = sa_bufs + buf * (kGgChunk * kGgBN) + row_in_tile;
-      for (int gg = 0; gg < gn; ++gg) {
+      float* da = sa_bufs + buf * (kGgChunk * kGgBM) + row_in_tile;
+      for (int gg = 0; gg < gn; ++gg)
         cp_async_4(db + gg * kGgBN, sbp + static_cast<int64_t>(gg) * p.sb_grp, cok ? 4u : 0u);
-        cp_async_4(da + gg * kGgBN, sap + static_cast<int64_t>(gg) * p.sa_grp, rok ? 4u : 0u);
-      }
+      if (sa_stager)
+        for (int gg = 0; gg < gn; ++gg)
+          cp_async_4(da + gg * kGgBM, sap + static_cast<int64_t>(gg) * p.sa_grp, rok ? 4u : 0u);
       cp_async_commit();
     };
     uint32_t gi = 0;
@@ -264,11 +280,11 @@ __global__ void __launch_bounds__(kGgThreads, 1)
           if (nt < p.num_tiles) stage_chunk(nt, ng0, buf ^ 1u);
         }
         const float* sb_chunk = sb_bufs + buf * (kGgChunk * kGgBN);
-        const float* sa_chunk = sa_bufs + buf * (kGgChunk * kGgBN);
+        const float* sa_chunk = sa_bufs + buf * (kGgChunk * kGgBM);
         const int gn = min(kGgChunk, ngroups - g0);
 #pragma unroll 1
         for (int gg = 0; gg < gn; ++gg, ++gi) {
-          const float sa = sa_chunk[gg * kGgBN + row_in_tile];
+          const float sa = sa_chunk[gg * kGgBM + row_in_tile];
           const uint32_t pb = gi % kGgPartials;
           if (!dead && !mbar_wait(&pfull[pb], (gi / kGgPartials) & 1u, kSiteGgPromote)) dead = true;
           dead = __any_sync(0xffffffffu, dead);
@@ -276,24 +292,24 @@ __global__ void __launch_bounds__(kGgThreads, 1)
           tc_fence_after();
           const float* sb_buf = sb_chunk + gg * kGgBN;
 #pragma unroll
-          for (int ch = 0; ch < kGgColsPerThread / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_cols + pb * 128u + ch * 32, r);
+          for (int ch = 0; ch < kGgColsPerThread / kGgLdCols; ++ch) {
+          uint32_t r[kGgLdCols];
+          tmem_ld_32x32b_x4(t_cols + pb * static_cast<uint32_t>(kGgBN) + ch * kGgLdCols, r);
           tmem_ld_wait();
-          reg_fence32(r);  // no use of r is scheduled above the wait
-          if (ch == kGgColsPerThread / 32 - 1) {
+          reg_fence4(r);  // no use of r is scheduled above the wait
+          if (ch == kGgColsPerThread / kGgLdCols - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&pempty[pb]);  // the partial is in registers: free it early
           }
-          const float4* sbv4 = reinterpret_cast<const float4*>(sb_buf + slice * kGgColsPerThread + ch * 32);
+          const float4* sbv4 = reinterpret_cast<const float4*>(sb_buf + slice * kGgColsPerThread + ch * kGgLdCols);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < kGgLdCols / 4; ++q) {
             const float4 sbq = sbv4[q];
 #pragma unroll
             for (int e = 0; e < 4; e += 2) {
               const int j = 4 * q + e;
-              const int jr = ch * 32 + j;  // index into run[]
+              const int jr = ch * kGgLdCols + j;  // index into run[]
               float2 a;
               if (QT == 0)
                 a = make_float2(__int2float_rn(static_cast<int>(r[j])), __int2float_rn(static_cast<int>(r[j + 1])));
