@@ -796,14 +796,20 @@ def measure_other_configs(pk: dict, reps: int = 20) -> dict:
         qt = halo.HALO_Q_INT8 if qname == "int8" else halo.HALO_Q_E4M3
         st = LayerStep(shapes, seed=4, device=torch.device("cuda"), qtype=qt, kinds=kinds)
         g = capture_step(st)
+        clk = None
         if wl == "llama70b_layer_fwd_bwd":
-            ts = _timed(g.replay, 10)
+            with ClockSampler(torch.cuda.current_device()) as sampler:
+                ts = _timed(g.replay, 20)
+            clk = sampler.summary()
         else:
             ts = _timed(g.replay, reps, flush)
         ms = med(ts)
         tops = st.ops_per_step() / (ms * 1e-3) / 1e12
         out.setdefault(wl, {})[qname] = {"ms_per_step": ms, "tops": tops, "frac_burst": tops / peak8,
                                          "target_frac": 0.60, "launches": st.launches_per_step()}
+        if clk is not None:
+            out[wl][qname]["clocks"] = clk
+            out[wl][qname]["ms_min_max"] = [min(ts), max(ts)]
         del g, st
         torch.cuda.synchronize()
     return out

@@ -358,12 +358,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       uint32_t ld_issued = 0, ld_par = 0;  // loads issued per stage, for the drain below
-      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+      int lt = 0;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++lt) {
         int tm, tn;
         gemm_tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
         const int b_row = tn * 256 + static_cast<int>(rank) * 128;
+        // Every pair takes its lt-th tile at about the same time, so the tiles
+        // of one pass over the grid share A panels with the pass before.  Odd
+        // passes walk K backwards: their first K blocks are the ones the
+        // previous pass read last, still in L2.  (The MMA loop accumulates in
+        // arrival order; INT8 sums are exact in any order.)
+        const bool reverse = (lt & 1) != 0;
         for (int kb = 0; kb < kblocks; ++kb) {
+          const int kpos = reverse ? kblocks - 1 - kb : kb;
           if (!mbar_wait(&empty[stage], phase ^ 1u, kSitePairProducer)) { ok = false; break; }
           note_load(ld_issued, ld_par, stage, phase);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
@@ -371,13 +379,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* a_dst = sA + stage * kPairABytes;
           uint8_t* b_dst = sB + stage * kPairBBytes;
           if (p.a_mn)
-            tma_load_2d_pair(a_dst, &tm_a, bar, a_row, kb * kGemmBK);
+            tma_load_2d_pair(a_dst, &tm_a, bar, a_row, kpos * kGemmBK);
           else
-            tma_load_2d_pair(a_dst, &tm_a, bar, kb * kGemmBK, a_row);
+            tma_load_2d_pair(a_dst, &tm_a, bar, kpos * kGemmBK, a_row);
           if (p.b_mn)
-            tma_load_2d_pair(b_dst, &tm_b, bar, b_row, kb * kGemmBK);
+            tma_load_2d_pair(b_dst, &tm_b, bar, b_row, kpos * kGemmBK);
           else
-            tma_load_2d_pair(b_dst, &tm_b, bar, kb * kGemmBK, b_row);
+            tma_load_2d_pair(b_dst, &tm_b, bar, kpos * kGemmBK, b_row);
           if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
         }
       }
