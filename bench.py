@@ -47,8 +47,8 @@ METRIC = "rotated-qGEMM TOPS & rotate+quant GB/s at Llama shapes vs B200 peak (1
 # GEMMs of the INT8 layer step, from one ncu capture, and the SHA-256 prefix of
 # the GEMM kernel source (csrc/qgemm.cuh) that capture ran.  The bench reports
 # the figure only while the source still hashes the same, null otherwise.
-GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER = 494.2e6
-GEMM_TRAFFIC_SOURCE_SHA = "86a812b144a4218c"
+GEMM_TRAFFIC_BYTES_PER_LAUNCH_INT8_LAYER = 462.3e6
+GEMM_TRAFFIC_SOURCE_SHA = "2eae0e678d021206"
 UNIT = "TOPS"
 BLK = 128
 # The sustained 8-bit denominator applies when the timed region lasts long
