@@ -535,6 +535,37 @@ def test_qgemm_grouped_parity(qtype, group, a_major, b_major, m, n, k):
 
 @pytest.mark.parametrize("qtype", [INT8, E4M3])
 @pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1)])
+def test_qgemm_grouped_many_tiles_sampled(qtype, group, a_major, b_major):
+    """4096 x 4000 x 1920: 512 tiles of 128 x 256 over 148 CTAs (each CTA runs
+    several tiles, the partial and scale-staging phases carry across them),
+    15 or 30 groups (a ragged last scale chunk), N not a multiple of 256 (the
+    last tile's second B box lies past the matrix).  Sampled rows and columns
+    against the oracle's grouped product of those rows and columns."""
+    m, n, k = 4096, 4000, 1920
+    a = _rand_codes(m, k, qtype, seed=91 + group)
+    b = _rand_codes(n, k, qtype, seed=92 + group)
+    sa = _group_scales(m, k // group, seed=93)
+    sb = _group_scales(n, k // group, seed=94)
+    sa_dev = _cuda(sa if a_major == 0 else sa.t().contiguous())
+    sb_dev = _cuda(sb if b_major == 0 else sb.t().contiguous())
+    c = halo.halo_qgemm_grouped(_cuda(_stored(a, a_major)), sa_dev, a_major, _cuda(_stored(b, b_major)), sb_dev,
+                                b_major, m, n, k, group, qtype, FP32)
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(95)
+    rows = torch.cat([torch.tensor([0, 127, 128, m - 1]), torch.randint(0, m, (28,), generator=g)])
+    cols = torch.cat([torch.tensor([0, 255, 256, 3839, 3840, n - 1]), torch.randint(0, n, (26,), generator=g)])
+    ref = oracle.gemm_grouped(a[rows].view(torch.uint8).numpy(), sa[rows].numpy(), b[cols].view(torch.uint8).numpy(),
+                              sb[cols].numpy(), group, qtype)
+    got = c.cpu()[rows][:, cols].numpy().astype(np.float64)
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+    st, site = halo.halo_device_error()
+    assert st == halo.HALO_OK, f"bounded wait ran out at site {site:#x}"
+
+
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("group", [64, 128])
 def test_linear_grouped_parity(qtype, group):
     m, n, k = 384, 320, 640
     x = inputs.activations(m, k, seed=71, device="cpu")
