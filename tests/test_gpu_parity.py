@@ -110,6 +110,36 @@ def test_qgemm_int8_bit_exact(a_major, b_major, m, n, k):
     np.testing.assert_array_equal(c.cpu().numpy(), acc.astype(np.float32))
 
 
+@pytest.mark.parametrize("qtype", [INT8, E4M3])
+@pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1), (0, 1)])
+def test_qgemm_long_k_two_passes_sampled(qtype, a_major, b_major):
+    """2048 x 4096 x 16384: 128 tiles of 256 x 256 over 74 SM pairs, so the
+    second pass over the grid walks K backwards (K >= 16384).  INT8 with unit
+    scales must still equal float32 of the exact integer sum; E4M3 within fp32
+    accumulation.  Sampled rows (both passes) and columns."""
+    m, n, k = 2048, 4096, 16384
+    a = _rand_codes(m, k, qtype, seed=81)
+    b = _rand_codes(n, k, qtype, seed=82)
+    ones_m = torch.ones(m, dtype=torch.float32, device="cuda")
+    ones_n = torch.ones(n, dtype=torch.float32, device="cuda")
+    c = halo.halo_qgemm(_cuda(_stored(a, a_major)), ones_m, a_major, _cuda(_stored(b, b_major)), ones_n, b_major,
+                        m, n, k, qtype, FP32)
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(83)
+    rows = torch.cat([torch.tensor([0, 255, 256, m - 1]), torch.randint(0, m, (28,), generator=g)])
+    cols = torch.cat([torch.tensor([0, 255, 256, n - 1]), torch.randint(0, n, (28,), generator=g)])
+    got = c.cpu()[rows][:, cols].numpy()
+    if qtype == INT8:
+        acc = oracle.gemm_i8(a[rows].numpy(), b[cols].numpy())
+        np.testing.assert_array_equal(got, acc.astype(np.float32))
+    else:
+        ref = oracle.gemm_e4m3(a[rows].view(torch.uint8).numpy(), b[cols].view(torch.uint8).numpy())
+        err = np.abs(got.astype(np.float64) - ref).max() / np.abs(ref).max()
+        assert err < 1e-5, err
+    st, site = halo.halo_device_error()
+    assert st == halo.HALO_OK, f"bounded wait ran out at site {site:#x}"
+
+
 @pytest.mark.parametrize("a_major,b_major", [(0, 0), (1, 1)])
 @pytest.mark.parametrize("otype", [FP32, BF16])
 def test_qgemm_e4m3_with_scales(a_major, b_major, otype):
