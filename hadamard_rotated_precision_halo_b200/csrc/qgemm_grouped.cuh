@@ -219,16 +219,16 @@ __global__ void __launch_bounds__(kGgThreads, 1)
     __syncwarp();
   } else {
     // Promotion.  A warp may only read tensor-memory lanes 32*(warp%4) .. +31:
-    // that quarter gives the tile rows, (warp - 2) / 4 the 32-column slice.
+    // that quarter gives the tile rows, (warp - 2) / 4 the 128-column half.
     const int quad = warp & 3;
-    const int slice = (warp - 2) >> 2;  // this thread's kGgColsPerThread-column slice
+    const int slice = (warp - 2) >> 2;  // this thread's kGgColsPerThread columns: 0 or 1
     const int row_in_tile = quad * 32 + lane;
     const int ngroups = p.k / p.group;
-    // Scale staging: the 128 threads of the first four promotion warps copy,
-    // for a chunk of kGgChunk groups, one column's s_b and one row's s_a per
-    // group into shared memory (warps 2-5 cover lane quarters 2, 3, 0, 1, so
-    // their rows are the tile's 128 rows).  The copies of the next chunk are
-    // issued as soon as a chunk starts and land while it is promoted.
+    // Scale staging: for a chunk of kGgChunk groups, each of the 256 promotion
+    // threads copies one column's s_b per group into shared memory, and the
+    // 128 threads of warps 2-5 (lane quarters 2, 3, 0, 1: the tile's 128 rows)
+    // one row's s_a.  The copies of the next chunk are issued as soon as a
+    // chunk starts and land while it is promoted.
     const bool sb_stager = (warp - 2) < kGgBN / 32;  // warps 2-9: one column each
     const bool sa_stager = (warp - 2) < 4;           // warps 2-5: one row each
     const bool stager = sb_stager;
