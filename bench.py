@@ -65,8 +65,11 @@ def gemm_source_sha() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def peaks(path: str = None):
+    """HBM copy GB/s and dense bf16 TFLOP/s (burst, sustained) measured on this
+    pool's B200s (MEASURED_PEAKS.json at the repository root), else the
+    fallback figures, saying which."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
@@ -74,6 +77,17 @@ def peaks():
                 "source": "measured"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_peak(pk: dict, region_s: float):
+    """The dense 8-bit denominator for the GEMM roofline: the measured bf16
+    figure times the nominal 8-bit : bf16 ratio (4.5 : 2.25), burst for a timed
+    region shorter than SUSTAINED_REGION_S, sustained (power-capped) otherwise.
+    Returns (peak, kind, burst, sustained)."""
+    burst, sustained = 2.0 * pk["bf16"], 2.0 * pk["bf16_sustained"]
+    if region_s >= SUSTAINED_REGION_S:
+        return sustained, "sustained", burst, sustained
+    return burst, "burst", burst, sustained
 
 
 # --------------------------------------------------------------------------- clocks
@@ -992,12 +1006,9 @@ def main():
     gemm_tops = step.gemm_ops() * args.steps / (gemm_ms * 1e-3) / 1e12
     rotq_gbs = step.rotq_bytes() * args.steps / (rotq_ms * 1e-3) / 1e9
     pk = peaks()
-    # INT8 / FP8 dense peak: the measured bf16 cuBLAS figure times the nominal
-    # 8-bit : bf16 ratio (4.5 : 2.25), burst or sustained by the timed region's length.
-    peak8_burst, peak8_sus = 2.0 * pk["bf16"], 2.0 * pk["bf16_sustained"]
     region_s = ms_total * 1e-3
-    sustained = region_s >= SUSTAINED_REGION_S
-    peak8 = peak8_sus if sustained else peak8_burst
+    peak8, peak_kind, peak8_burst, peak8_sus = gemm_peak(pk, region_s)
+    sustained = peak_kind == "sustained"
 
     def gbs(axis):  # 3 B per element (bf16 in, code out); both axes from one read: 4 B
         return (4 if axis == 2 else 3) * by_axis[axis][1] / max(by_axis[axis][0] * 1e-3, 1e-12) / 1e9
